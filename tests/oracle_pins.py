@@ -1,0 +1,250 @@
+"""Checks that pin the fp64 oracle to things other than itself.
+
+Each ``pin_*`` function takes a loaded oracle library handle and raises
+AssertionError when the oracle disagrees with what the TriAttention pages and
+the mathematics fix:
+
+* worked examples small enough to check by hand (``golden/hand_examples.json``);
+* the closed form the method rests on: with every query at its centre (R = 1,
+  so the norm term vanishes) the trigonometric score equals the mean over the
+  future offsets of the real dot product of the RoPE-rotated query centre and
+  the stored key, computed here from the textbook 2x2 rotation per band;
+* invariants: the score does not depend on the key positions once the stored
+  keys and t are fixed (positions cancel between un-rotation and distance);
+  moving t by c equals rotating the query centres by c; the norm term does
+  not change when a key band is rotated; z has mean 0 and variance 1 per
+  head; scaling every query statistic by c > 0 leaves z and the kept set alone;
+* brute force on tiny inputs: the kept set is the lexicographically smallest
+  of the B-subsets with the largest sum of max-z.
+
+The mutation test plants plausible mistakes in copies of the oracle and checks
+that each one trips at least one of these pins.
+"""
+from __future__ import annotations
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LAYOUTS = {"half": oracle.HALF, "interleaved": oracle.INTERLEAVED}
+
+
+def _bf16_bits(x):
+    """Round fp64 values to bf16 (round to nearest even) and return the bits."""
+    f = np.asarray(x, dtype=np.float32)
+    u = f.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return u.astype(np.uint16)
+
+
+def _bf16_value(bits):
+    return (np.asarray(bits, dtype=np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def _band_pairs(d, layout):
+    F = d // 2
+    if layout == oracle.HALF:
+        return [(f, f + F) for f in range(F)]
+    return [(2 * f, 2 * f + 1) for f in range(F)]
+
+
+def rope_rotate(x, m, base, layout):
+    """Textbook RoPE: rotate each band (a, b) of the real vector x by m * base^(-2f/d)."""
+    x = np.asarray(x, dtype=np.float64)
+    d = x.shape[-1]
+    out = x.copy()
+    for f, (a, b) in enumerate(_band_pairs(d, layout)):
+        th = m * base ** (-2.0 * f / d)
+        rot = np.array([[math.cos(th), -math.sin(th)], [math.sin(th), math.cos(th)]])
+        out[..., a], out[..., b] = (rot[0, 0] * x[..., a] + rot[0, 1] * x[..., b],
+                                    rot[1, 0] * x[..., a] + rot[1, 1] * x[..., b])
+    return out
+
+
+def _rand_unit(rng, d, G, N, layout, base, r_one=False):
+    F = d // 2
+    # the statistics enter as fp32 (as at the library boundary): draw them fp32-exact
+    q_mean = rng.standard_normal((G, d)).astype(np.float32).astype(np.float64)
+    pairs = _band_pairs(d, layout)
+    mag = np.stack([np.hypot(q_mean[:, a], q_mean[:, b]) for a, b in pairs], axis=1)
+    R = np.ones((G, F)) if r_one else rng.uniform(0.5, 1.0, (G, F))
+    q_norm = (mag / R).astype(np.float32).astype(np.float64)
+    R = R.astype(np.float32).astype(np.float64)
+    K = _bf16_bits(rng.standard_normal((N, d)) + rng.standard_normal(d))
+    pos = np.sort(rng.choice(4 * N + 64, N, replace=False)).astype(np.int32)
+    t = int(pos[-1]) + 1 + int(rng.integers(0, 5))
+    return q_mean, q_norm, R, K, pos, t
+
+
+def _expr(e):
+    return float(eval(e, {"__builtins__": {}}, {"math": math}))
+
+
+def pin_hand_examples(L):
+    with open(os.path.join(HERE, "golden", "hand_examples.json")) as fh:
+        g = json.load(fh)
+    for ex in g["scores"]:
+        K = _bf16_bits(np.array(ex["K"], dtype=np.float64))
+        assert np.array_equal(_bf16_value(K), np.array(ex["K"])), ex["name"]
+        s, _, _ = oracle.unit_scores(K, ex["pos"], ex["t"], ex["q_mean"], ex["q_norm"], ex["R"],
+                                     ex["offsets"], ex["base"], LAYOUTS[ex["layout"]], L=L)
+        want = np.array([_expr(e) for e in ex["expect"]])
+        assert np.allclose(s[:, 0], want, rtol=0, atol=1e-12), (ex["name"], s[:, 0], want)
+    for ex in g["zmax"]:
+        z, zm = oracle.zmax(np.array(ex["s"]), L=L)
+        assert np.allclose(z[0], [_expr(e) for e in ex["expect_z0"]], atol=1e-12), ex["name"]
+        assert np.allclose(zm, [_expr(e) for e in ex["expect_zmax"]], atol=1e-12), ex["name"]
+        for B, kept in ex["keep"].items():
+            got = oracle.select(zm, int(B), L=L)
+            assert got.tolist() == kept, (ex["name"], B, got, kept)
+
+
+def pin_rope_dot_closed_form(L, seed=0):
+    """R = 1: score == mean_delta RoPE(qbar, t + delta) . k~ (stored key), to 1e-9 of scale."""
+    rng = np.random.default_rng(seed)
+    for d, base, offsets in ((8, 1e4, [0]), (64, 1e4, [1 << i for i in range(11)]),
+                             (128, 1e6, [1 << i for i in range(17)])):
+        for layout in (oracle.HALF, oracle.INTERLEAVED):
+            G, N = 3, 17
+            q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base, r_one=True)
+            s, trig, norm = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets, base, layout, L=L)
+            kval = _bf16_value(K)
+            want = np.zeros((G, N))
+            for h in range(G):
+                for dl in offsets:
+                    qrot = rope_rotate(q_mean[h], t + dl, base, layout)
+                    want[h] += kval @ qrot
+                want[h] /= len(offsets)
+            scale = np.abs(want).max()
+            assert np.abs(norm).max() == 0.0
+            assert np.abs(s - want).max() <= 1e-9 * scale, (d, layout, np.abs(s - want).max(), scale)
+
+
+def pin_positions_cancel(L, seed=1):
+    """Fixed stored keys and t: moving the key positions must not change any score."""
+    rng = np.random.default_rng(seed)
+    for layout in (oracle.HALF, oracle.INTERLEAVED):
+        d, G, N, base = 128, 4, 23, 1e6
+        off = [1 << i for i in range(17)]
+        q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base)
+        s1, _, _ = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, off, base, layout, L=L)
+        pos2 = np.sort(rng.choice(t, N, replace=False)).astype(np.int32)
+        s2, _, _ = oracle.unit_scores(K, pos2, t, q_mean, q_norm, R, off, base, layout, L=L)
+        assert np.abs(s1 - s2).max() <= 1e-9 * np.abs(s1).max(), np.abs(s1 - s2).max()
+
+
+def pin_t_shift_is_query_rotation(L, seed=2):
+    """Score at t + c with centres qbar equals score at t with centres RoPE(qbar, c)."""
+    rng = np.random.default_rng(seed)
+    for layout in (oracle.HALF, oracle.INTERLEAVED):
+        d, G, N, base, c = 64, 2, 19, 1e4, 37
+        off = [1 << i for i in range(11)]
+        q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base)
+        s1, tr1, _ = oracle.unit_scores(K, pos, t + c, q_mean, q_norm, R, off, base, layout, L=L)
+        q_rot = np.stack([rope_rotate(q_mean[h], c, base, layout) for h in range(G)])
+        s2, tr2, _ = oracle.unit_scores(K, pos, t, q_rot, q_norm, R, off, base, layout, L=L)
+        # the rotated centres pass through fp32 at the interface: 1e-6 of scale
+        assert np.abs(tr1 - tr2).max() <= 1e-6 * np.abs(tr1).max()
+        assert np.abs(s1 - s2).max() <= 1e-6 * np.abs(s1).max()
+
+
+def pin_norm_rotation_invariant_and_linear(L, seed=3):
+    """The norm term ignores band rotations of the key and is linear in the weights."""
+    rng = np.random.default_rng(seed)
+    for layout in (oracle.HALF, oracle.INTERLEAVED):
+        d, G, N, base = 16, 2, 9, 1e4
+        q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base)
+        zero = np.zeros_like(q_mean)
+        _, tr, n1 = oracle.unit_scores(K, pos, t, zero, q_norm, R, [1, 2], base, layout, L=L)
+        assert np.abs(tr).max() == 0.0
+        # rotate every band of every key by a quarter turn: (a, b) -> (-b, a) is exact in bf16
+        K2 = K.copy()
+        for a, b in _band_pairs(d, layout):
+            K2[:, a] = K[:, b] ^ np.uint16(0x8000)
+            K2[:, b] = K[:, a]
+        _, _, n2 = oracle.unit_scores(K2, pos, t, zero, q_norm, R, [1, 2], base, layout, L=L)
+        assert np.abs(n1 - n2).max() <= 1e-12 * np.abs(n1).max()
+        # linearity in the weight (1 - R) E|q|
+        _, _, na = oracle.unit_scores(K, pos, t, zero, q_norm, np.zeros_like(R), [1], base, layout, L=L)
+        _, _, nb = oracle.unit_scores(K, pos, t, zero, q_norm, 0.75 * np.ones_like(R), [1], base, layout, L=L)
+        assert np.abs(nb - 0.25 * na).max() <= 1e-12 * np.abs(na).max()
+        # R = 1 removes it
+        _, _, nc = oracle.unit_scores(K, pos, t, zero, q_norm, np.ones_like(R), [1], base, layout, L=L)
+        assert np.abs(nc).max() == 0.0
+
+
+def pin_z_invariants(L, seed=4):
+    rng = np.random.default_rng(seed)
+    for G, N in ((1, 5), (4, 300), (8, 77)):
+        s = rng.standard_normal((G, N)) * rng.uniform(0.1, 50, (G, 1)) + rng.uniform(-9, 9, (G, 1))
+        z, zm = oracle.zmax(s, L=L)
+        assert np.abs(z.mean(axis=1)).max() <= 1e-12
+        assert np.abs((z * z).mean(axis=1) - 1.0).max() <= 1e-12
+        assert np.array_equal(zm, z.max(axis=0))
+        # flat head gives zero z
+        s2 = s.copy(); s2[0] = 3.25
+        z2, _ = oracle.zmax(s2, L=L)
+        assert np.all(z2[0] == 0.0)
+
+
+def pin_scale_invariance(L, seed=5):
+    """Scaling qbar and E|q| by c > 0 scales every score by c: z and the kept set do not move."""
+    rng = np.random.default_rng(seed)
+    d, G, N, base, B = 64, 4, 200, 1e4, 37
+    off = [1 << i for i in range(11)]
+    q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, oracle.HALF, base)
+    # keep 2.5 * stats exact in fp32: round the stats to 2^-10 steps first
+    q_mean = np.round(q_mean * 1024) / 1024
+    q_norm = np.round(q_norm * 1024) / 1024
+    V = K[::-1].copy()
+    a = oracle.prune_unit(K, V, pos, t, q_mean, q_norm, R, off, base, B, L=L)
+    b = oracle.prune_unit(K, V, pos, t, 2.5 * q_mean, 2.5 * q_norm, R, off, base, B, L=L)
+    assert np.abs(b["s"] - 2.5 * a["s"]).max() <= 1e-12 * np.abs(b["s"]).max()
+    assert np.abs(a["z"] - b["z"]).max() <= 1e-9
+    assert np.array_equal(a["kept"], b["kept"])
+
+
+def pin_select_brute_force(L, seed=6):
+    """Kept set == lexicographically smallest B-subset with the largest sum (integer zmax, many ties)."""
+    rng = np.random.default_rng(seed)
+    for trial in range(60):
+        N = int(rng.integers(1, 11))
+        B = int(rng.integers(1, 12))
+        zm = rng.integers(-3, 4, N).astype(np.float64)
+        got = oracle.select(zm, B, L=L).tolist()
+        M = min(N, B)
+        best = None
+        for sub in itertools.combinations(range(N), M):
+            key = (-sum(zm[list(sub)]), sub)
+            if best is None or key < best:
+                best = key
+        assert got == list(best[1]), (zm, B, got, best)
+
+
+def pin_compaction(L, seed=7):
+    rng = np.random.default_rng(seed)
+    d, G, N, base = 32, 2, 150, 1e4
+    q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, oracle.HALF, base)
+    V = _bf16_bits(rng.standard_normal((N, d)))
+    for B in (1, 40, 149, 150, 400):
+        r = oracle.prune_unit(K, V, pos, t, q_mean, q_norm, R, [1, 4], base, B, L=L)
+        kept = r["kept"]
+        assert len(kept) == min(N, B)
+        assert np.all(np.diff(kept) > 0)
+        assert np.array_equal(r["K"], K[kept]) and np.array_equal(r["V"], V[kept])
+        assert np.array_equal(r["pos"], pos[kept])
+        # kept keys dominate dropped keys (ties to the lower slot)
+        drop = np.setdiff1d(np.arange(N), kept)
+        if len(drop) and len(kept):
+            assert r["zmax"][kept].min() >= r["zmax"][drop].max()
+
+
+ALL_PINS = [pin_hand_examples, pin_rope_dot_closed_form, pin_positions_cancel,
+            pin_t_shift_is_query_rotation, pin_norm_rotation_invariant_and_linear,
+            pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction]

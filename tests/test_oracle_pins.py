@@ -1,0 +1,10 @@
+"""The fp64 oracle against hand-worked examples, closed forms, invariants and brute force."""
+import pytest
+
+import oracle
+import oracle_pins
+
+
+@pytest.mark.parametrize("pin", oracle_pins.ALL_PINS, ids=lambda f: f.__name__)
+def test_pin(pin):
+    pin(oracle.lib())
