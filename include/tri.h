@@ -1,0 +1,200 @@
+/*
+ * tri.h -- C ABI of the B200 (sm_100a) TriAttention KV-cache scoring-and-pruning pass.
+ *
+ * Pages cited (titles; sections as headed on each page):
+ *   [Deep-dive]  "TriAttention深度解析：用三角函数革命性压缩KV Cache，让长推理从「显存地狱」中脱困"
+ *                (chenxutan.com/d/2624)
+ *   [Stage]      "旋转舞台上的追光者——TriAttention如何用三角函数破解长文本推理的内存困局"
+ *                (zhichai.net/topic/177169654)
+ *   [10100]      the 10100.com article 127765992 on TriAttention (untitled extract)
+ *   [Summary]    "TriAttention：面向长文本推理的高效KV缓存压缩，2.5倍吞吐提升与10.7倍内存缩减"
+ *                (watermelonwater.tech)
+ *
+ * The pass, per unit = one (sequence s, layer l, KV head g) slice of the cache:
+ *   score   s_h(i) = mean_{delta in D} sum_f |qbar_f| |k_f| cos(omega_f (t + delta - p_i) + phi_f)
+ *                    + sum_f (1 - R_f) E|q_f| |k_f|
+ *           for each of the G query heads h that share KV head g
+ *           ([Stage] §TriAttention：把理论变成算法 items 1-2; [10100] §TriAttention方法;
+ *            offsets D of [Deep-dive] §3.3),
+ *   z/max   z-score each head over the unit's keys, max over the G heads
+ *           ([10100] §TriAttention方法; [Summary] §方案设计 item 4),
+ *   select  keep the B keys with the largest max-z, ties to the lower slot,
+ *   compact move the kept K, V and position rows, in their original order, to
+ *           slots 0..min(N,B)-1 of the same unit ([Deep-dive] §4 prune_kv_cache),
+ * run by the caller once every 128 generated tokens ([10100] §TriAttention方法;
+ * [Summary] §方案设计 item 4).
+ *
+ * Conventions for every entry point:
+ *   - Device pointers are plain CUDA device addresses of memory the caller owns.
+ *     The library never frees, resizes or retains them past the call.
+ *   - `stream` is a cudaStream_t passed as void*. Every launch goes on it;
+ *     calls return as soon as the work is enqueued (asynchronous).
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns TRI_EINVAL (or TRI_ESTATE / TRI_EUNSUPPORTED) and launches
+ *     nothing. Problems only the device can see (a length above the capacity,
+ *     a page id outside the pool, a wait that ran out) are recorded in the
+ *     context's device status word and read with tri_get_error; the affected
+ *     sequence is left untouched. Kernels never trap.
+ *   - A context is bound to one device and is not thread-safe: serialise calls
+ *     that share a context. Calls that share a context but run on different
+ *     streams must not overlap on the GPU (they share the status word and the
+ *     completion counter).
+ */
+#ifndef TRI_H_
+#define TRI_H_
+
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define TRI_API __attribute__((visibility("default")))
+#else
+#define TRI_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    TRI_OK = 0,
+    TRI_EINVAL = 1,       /* bad argument; nothing was launched */
+    TRI_ENOMEM = 2,       /* device or host allocation failed */
+    TRI_ECUDA = 3,        /* a CUDA runtime call failed */
+    TRI_ESTATE = 4,       /* no calibration statistics loaded */
+    TRI_EDEVICE = 5,      /* the device flagged bad input or a timed-out wait (tri_get_error) */
+    TRI_EUNSUPPORTED = 6  /* not an sm_100 device, or sizes beyond the on-chip limits */
+} tri_status;
+
+typedef enum {
+    TRI_ROPE_HALF = 0,        /* band f = dims (f, f + d/2): Qwen / NeoX rotary layout */
+    TRI_ROPE_INTERLEAVED = 1  /* band f = dims (2f, 2f + 1): GPT-J rotary layout */
+} tri_rope_layout;
+
+/* Device-side problem codes reported by tri_get_error in *detail_code. */
+enum {
+    TRI_DEV_NONE = 0,
+    TRI_DEV_LEN_GT_CAP = 1,   /* lens[s] < 0 or above the unit capacity */
+    TRI_DEV_BAD_PAGE = 2,     /* a block-table entry outside [0, n_pages) */
+    TRI_DEV_TIMEOUT = 3,      /* a bounded wait on an asynchronous copy gave up */
+    TRI_DEV_INTERNAL = 4      /* the selection did not produce exactly min(len, B) keys */
+};
+
+typedef struct tri_ctx tri_ctx;   /* opaque: device statistics, status word, counters */
+
+/*
+ * The cache one call works on. All pointers are device pointers owned by the caller.
+ *
+ * Dense layout (block_table == NULL):
+ *   K, V  bf16 [n_layers][batch][n_kv_heads][cap][head_dim]   (16-byte aligned)
+ *   pos   int32 [n_layers][batch][n_kv_heads][cap]            ascending within a unit
+ * Paged layout (block_table != NULL), one pool per layer, shared block table:
+ *   K, V  bf16 [n_layers][n_pages][n_kv_heads][page_size][head_dim]
+ *   pos   int32 [n_layers][n_pages][n_kv_heads][page_size]
+ *   block_table int32 [batch][max_pages]: logical page j of sequence s lives in
+ *         pool page block_table[s][j]; a unit's capacity is max_pages * page_size.
+ * lens      int32 [batch]: cached tokens of each sequence (same for every layer and
+ *           KV head), read only.
+ * lens_out  int32 [batch] or NULL: receives min(lens[s], budget) after tri_prune for
+ *           every sequence the device accepted (may alias lens). Pass NULL when a
+ *           cache is pruned in several layer chunks and update lens after the last.
+ * layer_begin, n_layers: the layers this call covers, indexing the loaded statistics;
+ *           the buffers above hold exactly these n_layers layers.
+ * n_kv_heads and head_dim come from the loaded statistics.
+ */
+typedef struct {
+    void *K;
+    void *V;
+    int32_t *pos;
+    const int32_t *lens;
+    int32_t *lens_out;
+    const int32_t *block_table;
+    int32_t batch;
+    int32_t cap;          /* dense: slots per unit; ignored when paged */
+    int32_t page_size;    /* paged: tokens per page, a multiple of 16; ignored when dense */
+    int32_t max_pages;    /* paged: block-table row length */
+    int32_t n_pages;      /* paged: pages in each layer's pool */
+    int32_t layer_begin;
+    int32_t n_layers;
+} tri_kv;
+
+/* Create a context on CUDA device `device` (must be compute capability 10.0).
+ * Allocates a few bytes of device memory (status word, completion counter). */
+TRI_API tri_status tri_create(tri_ctx **out, int device);
+
+/* Release the context and everything it allocated. NULL is accepted. */
+TRI_API tri_status tri_destroy(tri_ctx *ctx);
+
+/*
+ * Load calibration statistics (host fp32 arrays, copied; the caller keeps ownership).
+ *   q_mean       [n_layers][n_kv_heads*group][head_dim]  pre-RoPE query centre qbar, in the
+ *                same dim layout as the keys ([Deep-dive] §3.4; [Stage] item 1: E[q_f])
+ *   q_norm_mean  [n_layers][n_kv_heads*group][head_dim/2] E|q_f| per band ([Stage] item 2)
+ *   R            [n_layers][n_kv_heads*group][head_dim/2] concentration R_f = |E q_f| / E|q_f|
+ *                ([Stage] §破局之道)
+ *   offsets      [n_offsets] future offsets delta ([Deep-dive] §3.3: 1, 2, 4, ..., 2^16)
+ * Query head h belongs to KV head h / group. head_dim in {64, 128}; group in {1, 2, 4, 8};
+ * rope_base > 0; all values finite. The per-band constants (omega_f, the offset average
+ * A_f = mean_delta e^{i omega_f delta}, qbar_f * A_f and (1 - R_f) E|q_f|) are formed
+ * here in fp64. Replaces any statistics loaded before. Synchronous.
+ */
+TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads, int group, int head_dim,
+                              double rope_base, tri_rope_layout layout,
+                              const float *q_mean, const float *q_norm_mean, const float *R,
+                              const int64_t *offsets, int n_offsets);
+
+/*
+ * Score every cached key and prune each unit to its top `budget` keys, in place.
+ *   t       int32 [batch] device: current query position of each sequence; the
+ *           future queries are at t + delta. Positions in the cache must be < t.
+ *   budget  B >= 1 keys kept per unit.
+ * After the call (in stream order) slots [0, min(len, B)) of every unit hold the kept
+ * K, V and position rows in ascending original order; slots at or beyond that are
+ * left as they were (reclaiming them is the caller's business); units with len <= B
+ * are not touched at all. lens_out receives the new lengths.
+ */
+TRI_API tri_status tri_prune(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream);
+
+/*
+ * Debug / parity entry: score without pruning.
+ *   raw   float [n_layers][batch][n_kv_heads*group][cap_u] or NULL: s_h(i) per query head
+ *   zmax  float [n_layers][batch][n_kv_heads][cap_u] or NULL: max over the group of z_h(i)
+ * where cap_u is cap (dense) or max_pages*page_size (paged), indexed by logical slot.
+ * Slots at or beyond lens[s] are not written. The cache is not modified; lens_out is ignored.
+ */
+TRI_API tri_status tri_score(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, float *raw, float *zmax,
+                     void *stream);
+
+/*
+ * Synchronise `stream`, read and clear the context's device status word.
+ * Returns TRI_OK, or TRI_EDEVICE with the first problem's code (TRI_DEV_*) and the
+ * unit index u = (layer_in_call * batch + s) * n_kv_heads + g it was seen on
+ * (either out-pointer may be NULL).
+ */
+TRI_API tri_status tri_get_error(tri_ctx *ctx, void *stream, int32_t *detail_code, int64_t *detail_unit);
+
+/*
+ * Launch-shape override for measurement and tests (not part of the paper's pass).
+ *   cluster_size      CTAs that share one unit: 1, 2, 4, 8 or 16; 0 = automatic
+ *                     (the smallest that holds the unit's scores on chip while giving
+ *                     the GPU at least two CTAs per SM).
+ *   buffers_per_warp  key-streaming buffers per warp, 1..4; 0 = automatic (2).
+ * Sizes that do not fit on chip with the requested shape make tri_prune / tri_score
+ * return TRI_EUNSUPPORTED.
+ */
+TRI_API tri_status tri_set_tuning(tri_ctx *ctx, int cluster_size, int buffers_per_warp);
+
+/* Text of the last host-side failure on this context (the CUDA error and the call that
+ * returned it), or an empty string. Valid until the next call on the context. */
+TRI_API const char *tri_last_error(tri_ctx *ctx);
+
+/* Static, human-readable name of a status. */
+TRI_API const char *tri_status_str(tri_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+TRI_API int tri_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRI_H_ */

@@ -1,0 +1,448 @@
+// tri_api.cu -- host side of the C ABI declared in include/tri.h.
+//
+// The statistics loader follows [Deep-dive] §3.4 (offline calibration: load the per-head
+// query statistics once) and folds the future-offset average of [Deep-dive] §3.3 into one
+// complex constant per band: mean_delta e^{i omega_f (t + delta)} = A_f e^{i omega_f t} with
+// A_f = mean_delta e^{i omega_f delta}. Everything that depends on t is formed on the device
+// (the phase e^{i omega_f t} in fp64) so that a call never waits on the host.
+//
+//   [Deep-dive]  "TriAttention深度解析：用三角函数革命性压缩KV Cache，让长推理从「显存地狱」中脱困"
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tri.h"
+#include "tri_kernel.cuh"
+
+struct tri_ctx {
+    int device = -1;
+    int sm_count = 0;
+    int max_smem_optin = 0;
+    // statistics
+    bool loaded = false;
+    int L = 0, Hkv = 0, G = 0, D = 0, layout = 0;
+    double *d_omega = nullptr;
+    double2 *d_Qc = nullptr;
+    float *d_w = nullptr;
+    // device bookkeeping
+    unsigned long long *d_status = nullptr;
+    unsigned int *d_counter = nullptr;
+    int32_t *d_seq_bad = nullptr;
+    int seq_bad_cap = 0;
+    // tuning (0 = automatic)
+    int tune_cs = 0;
+    int tune_nslot = 0;
+    // text of the last failure seen on the host (CUDA error name and the call that failed)
+    char last_error[256] = {0};
+};
+
+namespace {
+
+using KernelFn = void (*)(const tri::Args);
+
+template <int D, int G, int LAYOUT>
+KernelFn kernel_of() {
+    return &tri::tri_fused_kernel<D, G, LAYOUT>;
+}
+
+KernelFn pick_kernel(int D, int G, int layout) {
+#define TRI_CASE(DD, GG)                                                               \
+    if (D == DD && G == GG) return layout == 0 ? kernel_of<DD, GG, 0>() : kernel_of<DD, GG, 1>();
+    TRI_CASE(64, 1) TRI_CASE(64, 2) TRI_CASE(64, 4) TRI_CASE(64, 8)
+    TRI_CASE(128, 1) TRI_CASE(128, 2) TRI_CASE(128, 4) TRI_CASE(128, 8)
+#undef TRI_CASE
+    return nullptr;
+}
+
+bool finite_all(const float *p, size_t n) {
+    for (size_t i = 0; i < n; ++i)
+        if (!std::isfinite(p[i])) return false;
+    return true;
+}
+
+void free_stats(tri_ctx *c) {
+    cudaFree(c->d_omega);
+    cudaFree(c->d_Qc);
+    cudaFree(c->d_w);
+    c->d_omega = nullptr;
+    c->d_Qc = nullptr;
+    c->d_w = nullptr;
+    c->loaded = false;
+}
+
+// Device memory check: a pointer the runtime does not know as device or managed memory
+// is rejected before anything is launched.
+bool is_device_ptr(const void *p) {
+    if (!p) return false;
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return at.type == cudaMemoryTypeDevice || at.type == cudaMemoryTypeManaged;
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Remember what failed, clear the runtime's sticky-free error state and map to a status.
+tri_status cuda_fail(tri_ctx *c, cudaError_t e, const char *what, tri_status st = TRI_ECUDA) {
+    if (c) {
+        std::snprintf(c->last_error, sizeof c->last_error, "%s: %s (%s)", what, cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+    }
+    cudaGetLastError();
+    return st;
+}
+
+struct Plan {
+    int cs = 0, nslot = 0, kpc = 0;
+    size_t smem = 0;
+};
+
+std::mutex g_attr_mu;
+
+cudaError_t prepare_kernel(KernelFn fn, int max_optin) {
+    // Opting in to the full shared-memory carve-out and to 16-CTA clusters is a property
+    // of the kernel function, set once per process.
+    static std::vector<KernelFn> done;
+    std::lock_guard<std::mutex> lk(g_attr_mu);
+    if (std::find(done.begin(), done.end(), fn) != done.end()) return cudaSuccess;
+    cudaFuncAttributes fa;
+    cudaError_t e = cudaFuncGetAttributes(&fa, fn);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             max_optin - (int)fa.sharedSizeBytes);
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+    done.push_back(fn);
+    return cudaSuccess;
+}
+
+// Pick the cluster size: the smallest that fits the unit's scores on chip and still gives
+// the GPU at least two CTAs per SM to schedule, else the largest that fits.
+tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Plan *out) {
+    cudaFuncAttributes fa;
+    cudaError_t fe = cudaFuncGetAttributes(&fa, fn);
+    if (fe != cudaSuccess) return cuda_fail(c, fe, "cudaFuncGetAttributes");
+    const size_t budget = (size_t)c->max_smem_optin - fa.sharedSizeBytes;
+    const int nslot = c->tune_nslot > 0 ? c->tune_nslot : 2;
+    Plan best;
+    for (int cs = 1; cs <= tri::kMaxCluster; cs *= 2) {
+        if (c->tune_cs > 0 && cs != c->tune_cs) continue;
+        const long long kpc = ((long long)(cap_u + cs - 1) / cs + 31) / 32 * 32;
+        if (kpc > 32768) continue;
+        const tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
+        if (Ly.total > budget || Ly.stage_rows < 16) continue;
+        // the cluster must be schedulable with this much shared memory per CTA
+        {
+            cudaLaunchConfig_t cfg;
+            std::memset(&cfg, 0, sizeof cfg);
+            cfg.gridDim = dim3((unsigned)cs);
+            cfg.blockDim = dim3(tri::kThreads);
+            cfg.dynamicSmemBytes = Ly.total;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = (unsigned)cs;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int nclusters = 0;
+            const cudaError_t oe = cudaOccupancyMaxActiveClusters(&nclusters, fn, &cfg);
+            if (oe != cudaSuccess) {
+                cuda_fail(c, oe, "cudaOccupancyMaxActiveClusters");
+                continue;
+            }
+            if (nclusters < 1) continue;
+        }
+        Plan p;
+        p.cs = cs;
+        p.nslot = nslot;
+        p.kpc = (int)kpc;
+        p.smem = Ly.total;
+        best = p;
+        if (n_units * cs >= 2LL * c->sm_count) break;
+    }
+    if (best.cs == 0) return TRI_EUNSUPPORTED;
+    *out = best;
+    return TRI_OK;
+}
+
+tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
+               int mode, void *stream) {
+    if (!c || !kv || !t) return TRI_EINVAL;
+    if (!c->loaded) return TRI_ESTATE;
+    if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
+        return TRI_EINVAL;
+    const bool paged = kv->block_table != nullptr;
+    long long cap_u;
+    if (paged) {
+        if (kv->page_size < 16 || kv->page_size % 16 != 0 || kv->max_pages < 1 || kv->n_pages < 1)
+            return TRI_EINVAL;
+        cap_u = (long long)kv->page_size * kv->max_pages;
+    } else {
+        if (kv->cap < 1) return TRI_EINVAL;
+        cap_u = kv->cap;
+    }
+    if (cap_u > (1LL << 30)) return TRI_EUNSUPPORTED;
+    if (mode == tri::kModePrune) {
+        if (budget < 1) return TRI_EINVAL;
+        if (!kv->K || !kv->V || !kv->pos || !kv->lens) return TRI_EINVAL;
+        if (!aligned(kv->K, 16) || !aligned(kv->V, 16) || !aligned(kv->pos, 4)) return TRI_EINVAL;
+        if (!is_device_ptr(kv->K) || !is_device_ptr(kv->V) || !is_device_ptr(kv->pos)) return TRI_EINVAL;
+        if (kv->lens_out && (!is_device_ptr(kv->lens_out) || !aligned(kv->lens_out, 4))) return TRI_EINVAL;
+    } else {
+        if (!kv->K || !kv->lens) return TRI_EINVAL;
+        if (!aligned(kv->K, 16) || !is_device_ptr(kv->K)) return TRI_EINVAL;
+        if (raw && (!aligned(raw, 4) || !is_device_ptr(raw))) return TRI_EINVAL;
+        if (zmax && (!aligned(zmax, 4) || !is_device_ptr(zmax))) return TRI_EINVAL;
+    }
+    if (!is_device_ptr(kv->lens) || !is_device_ptr(t) || !aligned(kv->lens, 4) || !aligned(t, 4))
+        return TRI_EINVAL;
+    if (paged && (!is_device_ptr(kv->block_table) || !aligned(kv->block_table, 4))) return TRI_EINVAL;
+
+    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
+    if (n_units * tri::kMaxCluster > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+
+    KernelFn fn = pick_kernel(c->D, c->G, c->layout);
+    if (!fn) return TRI_EUNSUPPORTED;
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+    ce = prepare_kernel(fn, c->max_smem_optin);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute");
+    Plan plan;
+    tri_status st = plan_launch(c, fn, (int)cap_u, n_units, &plan);
+    if (st != TRI_OK) return st;
+
+    const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
+    if (finalize && kv->batch > c->seq_bad_cap) {
+        cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
+        c->d_seq_bad = nullptr;
+        c->seq_bad_cap = 0;
+        if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ENOMEM;
+        if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ECUDA;
+        c->seq_bad_cap = kv->batch;
+    }
+
+    tri::Args a;
+    std::memset(&a, 0, sizeof a);
+    a.K = static_cast<uint16_t *>(kv->K);
+    a.V = static_cast<uint16_t *>(kv->V);
+    a.pos = kv->pos;
+    a.lens = kv->lens;
+    a.lens_out = finalize ? kv->lens_out : nullptr;
+    a.block_table = kv->block_table;
+    a.t = t;
+    a.batch = kv->batch;
+    a.n_kv = c->Hkv;
+    a.cap_u = (int)cap_u;
+    a.paged = paged ? 1 : 0;
+    a.page_size = paged ? kv->page_size : 0;
+    a.max_pages = paged ? kv->max_pages : 0;
+    a.n_pages = paged ? kv->n_pages : 0;
+    a.layer_begin = kv->layer_begin;
+    a.budget = mode == tri::kModePrune ? budget : 0x7fffffff;
+    a.omega = c->d_omega;
+    a.Qc = c->d_Qc;
+    a.w = c->d_w;
+    a.raw = raw;
+    a.zmax = zmax;
+    a.mode = mode;
+    a.cs = plan.cs;
+    a.kpc_max = plan.kpc;
+    a.nslot = plan.nslot;
+    a.status = c->d_status;
+    a.counter = c->d_counter;
+    a.seq_bad = finalize ? c->d_seq_bad : nullptr;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)(n_units * plan.cs));
+    cfg.blockDim = dim3(tri::kThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)plan.cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ce = cudaLaunchKernelEx(&cfg, fn, a);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx");
+    return TRI_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+tri_status tri_create(tri_ctx **out, int device) {
+    if (!out) return TRI_EINVAL;
+    *out = nullptr;
+    int n = 0;
+    if (cudaGetDeviceCount(&n) != cudaSuccess) {
+        cudaGetLastError();
+        return TRI_ECUDA;
+    }
+    if (device < 0 || device >= n) return TRI_EINVAL;
+    cudaDeviceProp p;
+    if (cudaGetDeviceProperties(&p, device) != cudaSuccess) return TRI_ECUDA;
+    if (p.major != 10) return TRI_EUNSUPPORTED;
+    if (cudaSetDevice(device) != cudaSuccess) return TRI_ECUDA;
+    tri_ctx *c = new (std::nothrow) tri_ctx;
+    if (!c) return TRI_ENOMEM;
+    c->device = device;
+    c->sm_count = p.multiProcessorCount;
+    c->max_smem_optin = (int)p.sharedMemPerBlockOptin;
+    if (cudaMalloc(&c->d_status, sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMalloc(&c->d_counter, sizeof(unsigned int)) != cudaSuccess) {
+        tri_destroy(c);
+        return TRI_ENOMEM;
+    }
+    if (cudaMemset(c->d_status, 0, sizeof(unsigned long long)) != cudaSuccess ||
+        cudaMemset(c->d_counter, 0, sizeof(unsigned int)) != cudaSuccess) {
+        tri_destroy(c);
+        return TRI_ECUDA;
+    }
+    *out = c;
+    return TRI_OK;
+}
+
+tri_status tri_destroy(tri_ctx *c) {
+    if (!c) return TRI_OK;
+    if (c->device >= 0) cudaSetDevice(c->device);
+    free_stats(c);
+    cudaFree(c->d_status);
+    cudaFree(c->d_counter);
+    cudaFree(c->d_seq_bad);
+    delete c;
+    return TRI_OK;
+}
+
+tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int group, int head_dim,
+                              double rope_base, tri_rope_layout layout, const float *q_mean,
+                              const float *q_norm_mean, const float *R, const int64_t *offsets,
+                              int n_offsets) {
+    if (!c) return TRI_EINVAL;
+    if (n_layers < 1 || n_kv_heads < 1 || n_offsets < 1) return TRI_EINVAL;
+    if (head_dim != 64 && head_dim != 128) return TRI_EINVAL;
+    if (group != 1 && group != 2 && group != 4 && group != 8) return TRI_EINVAL;
+    if (!(rope_base > 0.0) || !std::isfinite(rope_base)) return TRI_EINVAL;
+    if (layout != TRI_ROPE_HALF && layout != TRI_ROPE_INTERLEAVED) return TRI_EINVAL;
+    if (!q_mean || !q_norm_mean || !R || !offsets) return TRI_EINVAL;
+    const int D = head_dim, F = D / 2, Hq = n_kv_heads * group;
+    const size_t nq = (size_t)n_layers * Hq * D, nb = (size_t)n_layers * Hq * F;
+    if (!finite_all(q_mean, nq) || !finite_all(q_norm_mean, nb) || !finite_all(R, nb)) return TRI_EINVAL;
+
+    // fp64 constants: omega_f = base^(-2f/d) and the offset average A_f
+    std::vector<double> omega(F);
+    std::vector<double> Are(F), Aim(F);
+    for (int f = 0; f < F; ++f) {
+        omega[f] = std::pow(rope_base, -2.0 * (double)f / (double)D);
+        double sr = 0.0, si = 0.0;
+        for (int j = 0; j < n_offsets; ++j) {
+            const double ang = omega[f] * (double)offsets[j];
+            sr += std::cos(ang);
+            si += std::sin(ang);
+        }
+        Are[f] = sr / n_offsets;
+        Aim[f] = si / n_offsets;
+    }
+    std::vector<double2> Qc(nb);
+    std::vector<float> w(nb);
+    for (size_t lh = 0; lh < (size_t)n_layers * Hq; ++lh) {
+        const float *q = q_mean + lh * D;
+        for (int f = 0; f < F; ++f) {
+            const int dre = layout == TRI_ROPE_HALF ? f : 2 * f;
+            const int dim = layout == TRI_ROPE_HALF ? f + F : 2 * f + 1;
+            const double qr = q[dre], qi = q[dim];
+            Qc[lh * F + f] = make_double2(qr * Are[f] - qi * Aim[f], qr * Aim[f] + qi * Are[f]);
+            w[lh * F + f] = (float)((1.0 - (double)R[lh * F + f]) * (double)q_norm_mean[lh * F + f]);
+        }
+    }
+    if (cudaSetDevice(c->device) != cudaSuccess) return TRI_ECUDA;
+    free_stats(c);
+    if (cudaMalloc(&c->d_omega, sizeof(double) * F) != cudaSuccess ||
+        cudaMalloc(&c->d_Qc, sizeof(double2) * nb) != cudaSuccess ||
+        cudaMalloc(&c->d_w, sizeof(float) * nb) != cudaSuccess) {
+        free_stats(c);
+        return TRI_ENOMEM;
+    }
+    if (cudaMemcpy(c->d_omega, omega.data(), sizeof(double) * F, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->d_Qc, Qc.data(), sizeof(double2) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->d_w, w.data(), sizeof(float) * nb, cudaMemcpyHostToDevice) != cudaSuccess) {
+        free_stats(c);
+        return TRI_ECUDA;
+    }
+    c->L = n_layers;
+    c->Hkv = n_kv_heads;
+    c->G = group;
+    c->D = D;
+    c->layout = layout;
+    c->loaded = true;
+    return TRI_OK;
+}
+
+tri_status tri_prune(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
+    return run(c, kv, t, budget, nullptr, nullptr, tri::kModePrune, stream);
+}
+
+tri_status tri_score(tri_ctx *c, const tri_kv *kv, const int32_t *t, float *raw, float *zmax, void *stream) {
+    return run(c, kv, t, 0, raw, zmax, tri::kModeScore, stream);
+}
+
+tri_status tri_set_tuning(tri_ctx *c, int cluster_size, int buffers_per_warp) {
+    if (!c) return TRI_EINVAL;
+    if (cluster_size != 0 && cluster_size != 1 && cluster_size != 2 && cluster_size != 4 &&
+        cluster_size != 8 && cluster_size != 16)
+        return TRI_EINVAL;
+    if (buffers_per_warp < 0 || buffers_per_warp > 4) return TRI_EINVAL;
+    c->tune_cs = cluster_size;
+    c->tune_nslot = buffers_per_warp;
+    return TRI_OK;
+}
+
+tri_status tri_get_error(tri_ctx *c, void *stream, int32_t *detail_code, int64_t *detail_unit) {
+    if (detail_code) *detail_code = 0;
+    if (detail_unit) *detail_unit = -1;
+    if (!c) return TRI_EINVAL;
+    if (cudaSetDevice(c->device) != cudaSuccess) return TRI_ECUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TRI_ECUDA;
+    unsigned long long v = 0;
+    if (cudaMemcpy(&v, c->d_status, sizeof v, cudaMemcpyDeviceToHost) != cudaSuccess) return TRI_ECUDA;
+    if (v == 0) return TRI_OK;
+    if (cudaMemset(c->d_status, 0, sizeof v) != cudaSuccess) return TRI_ECUDA;
+    if (detail_code) *detail_code = (int32_t)(v >> 32);
+    if (detail_unit) *detail_unit = (int64_t)(uint32_t)(v & 0xffffffffu);
+    return TRI_EDEVICE;
+}
+
+const char *tri_last_error(tri_ctx *c) {
+    if (!c) return "no context";
+    return c->last_error;
+}
+
+const char *tri_status_str(tri_status s) {
+    switch (s) {
+        case TRI_OK: return "TRI_OK";
+        case TRI_EINVAL: return "TRI_EINVAL: invalid argument";
+        case TRI_ENOMEM: return "TRI_ENOMEM: allocation failed";
+        case TRI_ECUDA: return "TRI_ECUDA: CUDA runtime error";
+        case TRI_ESTATE: return "TRI_ESTATE: no calibration statistics loaded";
+        case TRI_EDEVICE: return "TRI_EDEVICE: the device flagged a problem";
+        case TRI_EUNSUPPORTED: return "TRI_EUNSUPPORTED: unsupported device or size";
+    }
+    return "unknown tri_status";
+}
+
+int tri_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,940 @@
+// tri_kernel.cuh -- the fused TriAttention scoring-and-pruning kernel for sm_100a.
+//
+// Pages cited (titles; sections as headed on each page):
+//   [Deep-dive]  "TriAttention深度解析：用三角函数革命性压缩KV Cache，让长推理从「显存地狱」中脱困"
+//   [Stage]      "旋转舞台上的追光者——TriAttention如何用三角函数破解长文本推理的内存困局"
+//   [10100]      the 10100.com article 127765992 on TriAttention
+//   [Summary]    "TriAttention：面向长文本推理的高效KV缓存压缩，2.5倍吞吐提升与10.7倍内存缩减"
+//
+// One thread-block cluster owns one unit (sequence s, layer l, KV head g) and runs the
+// whole pass on it without a round trip through HBM:
+//
+//   prologue  C_{h,f} = (qbar_{h,f} A_f) e^{i omega_f t}, with A_f = mean_delta e^{i omega_f delta}
+//             (fp64 phase, rounded to fp32 once). Because the stored key is post-RoPE,
+//             mean_delta |qbar_f||k_f| cos(omega_f (t+delta-p) + arg qbar_f - arg k_f)
+//             = Re(C_f conj(k~_f)), so the trigonometric series of [Stage]
+//             §TriAttention：把理论变成算法 item 1, averaged over the offsets of [Deep-dive] §3.3,
+//             becomes one dot product per key and head; positions drop out.
+//   score     per key: s_h = sum_j c_{h,j} k~_j + sum_f w_{h,f} |k~_f|, w = (1 - R) E|q|
+//             ([Stage] item 2 with the (1 - R) weight of [10100] §TriAttention方法). Keys
+//             stream from HBM by TMA bulk copies (cp.async.bulk, mbarrier completion)
+//             into per-warp double buffers; each key is split over LPK lanes, every lane
+//             keeps its slice of the coefficients in registers and accumulates with
+//             packed fp32x2 FMAs; a reduce-scatter over the lanes finishes the G heads.
+//             Scores stay in shared memory.
+//   z / max   per head: mean and population std over all of the unit's keys (fp64 sums
+//             exchanged between the cluster's CTAs through distributed shared memory),
+//             z = (s - mu) / sigma (0 for a flat head), max over the G heads
+//             ([10100] §TriAttention方法; [Summary] §方案设计 item 4).
+//   select    top-B by max-z: four 8-bit radix passes over an order-preserving uint32
+//             image of the fp32 value, histograms merged across the cluster; exact ties
+//             at the threshold go to the lower slot.
+//   compact   in-place stable gather of the kept K/V/position rows to slots [0, B)
+//             ([Deep-dive] §4 prune_kv_cache: top-k then sort). Destinations are taken in
+//             rounds in ascending order; in each round every CTA first copies its
+//             sources into shared memory (cp.async), the cluster synchronises, then all
+//             CTAs write. Since a kept row never moves to a higher slot, no round can
+//             overwrite a row that this or a later round still has to read.
+#pragma once
+
+#include <cooperative_groups.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tri {
+
+namespace cg = cooperative_groups;
+
+constexpr int kStageRows = 16;      // rows per TMA bulk copy (one copy never crosses a page)
+constexpr int kBins = 256;          // radix digit width: 8 bits
+constexpr int kWarps = 8;           // warps per CTA
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxCluster = 16;
+constexpr int kModePrune = 0;
+constexpr int kModeScore = 1;
+constexpr int kDevLenGtCap = 1;
+constexpr int kDevBadPage = 2;
+constexpr int kDevTimeout = 3;
+constexpr int kDevInternal = 4;
+constexpr long long kWaitLimit = 1ll << 22;   // bounded mbarrier polls (with backoff: ~1 s)
+
+struct Args {
+    uint16_t *K;                 // bf16 bits
+    uint16_t *V;
+    int32_t *pos;
+    const int32_t *lens;
+    int32_t *lens_out;
+    const int32_t *block_table;
+    const int32_t *t;
+    int batch, n_kv, cap_u;
+    int paged, page_size, max_pages, n_pages;
+    int layer_begin;
+    int budget;
+    const double *omega;         // [F]
+    const double2 *Qc;           // [L][Hq][F]  qbar * A
+    const float *w;              // [L][Hq][F]  (1 - R) E|q|
+    float *raw;                  // score mode outputs (or null)
+    float *zmax;
+    int mode;
+    int cs;                      // cluster size (CTAs per unit)
+    int kpc_max;                 // key capacity of one CTA (multiple of 32)
+    int nslot;                   // TMA buffers per warp
+    unsigned long long *status;  // first device-detected problem
+    unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
+    int32_t *seq_bad;            // [batch] sequences the device refused this call
+};
+
+// Per-CTA values other CTAs of the cluster read through distributed shared memory.
+struct Xch {
+    double sum[8];
+    double m2[8];
+    float mn[8];
+    float mx[8];
+    int ties;
+    int kept;
+    int fail;
+    int pad;
+};
+
+struct Layout {
+    unsigned sc, ring, coef_t, coef_w, phase, whist, bhist, ghist, lmask, gmask, gpre, xch, misc,
+        srcidx, bars, total;
+    int stage_rows;    // compaction rows per CTA per round
+    unsigned regionA;  // bytes of sc + ring (reused as the compaction stage)
+};
+
+__host__ __device__ inline unsigned align_up(unsigned x, unsigned a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline Layout make_layout(int D, int G, int nslot, int kpc, int cs) {
+    Layout L;
+    unsigned o = 0;
+    const int F = D / 2;
+    const int nwl = kpc / 32;
+    L.sc = o;
+    o = align_up(o + (unsigned)kpc * G * 4u, 128);
+    L.ring = o;
+    o = align_up(o + (unsigned)kWarps * nslot * kStageRows * D * 2u, 128);
+    L.regionA = o;
+    const unsigned row_bytes = (unsigned)D * 2u * 2u + 4u;
+    int S = (int)(L.regionA / row_bytes);
+    S = S / 16 * 16;
+    L.stage_rows = S;
+    L.coef_t = o;
+    o = align_up(o + (unsigned)G * D * 4u, 16);
+    L.coef_w = o;
+    o = align_up(o + (unsigned)G * F * 4u, 16);
+    L.phase = o;
+    o = align_up(o + (unsigned)F * 16u, 16);
+    L.whist = o;
+    o = align_up(o + (unsigned)kWarps * kBins * 4u, 16);
+    L.bhist = o;
+    o = align_up(o + 2u * kBins * 4u, 16);
+    L.ghist = o;
+    o = align_up(o + (unsigned)kBins * 4u, 16);
+    L.lmask = o;
+    o = align_up(o + (unsigned)nwl * 4u, 16);
+    L.gmask = o;
+    o = align_up(o + (unsigned)cs * nwl * 4u, 16);
+    L.gpre = o;
+    o = align_up(o + ((unsigned)cs * nwl + 1u) * 4u, 16);
+    L.xch = o;
+    o = align_up(o + sizeof(Xch), 16);
+    L.misc = o;  // block-reduction scratch: kWarps * 8 doubles + broadcast words
+    o = align_up(o + (unsigned)kWarps * 8u * 8u + 64u * 4u + 8u * 16u, 16);
+    L.srcidx = o;
+    o = align_up(o + (unsigned)(S > 0 ? S : 1) * 4u, 16);
+    L.bars = o;
+    o = align_up(o + (unsigned)kWarps * nslot * 8u, 16);
+    L.total = o;
+    return L;
+}
+
+// ---------------------------------------------------------------------------------
+// PTX helpers
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ unsigned smem_u32(const void *p) {
+    return (unsigned)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, unsigned count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_init_fence() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
+    unsigned ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: returns false if the phase did not complete within the poll limit.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
+    for (long long i = 0; i < kWaitLimit; ++i) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if (i > 64) __nanosleep(256);
+    }
+    return false;
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 1-D bulk copy global -> shared, completion signalled on an mbarrier (no multicast).
+__device__ __forceinline__ void tma_load_1d(void *dst_smem, const void *src_gmem, unsigned bytes,
+                                            uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async4(void *dst_smem, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
+// acc += a * b on two fp32 lanes at once (sm_100 packed FMA).
+__device__ __forceinline__ void ffma2(float2 &acc, float2 a, float2 b) {
+    unsigned long long A, B, C;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
+    asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(acc.x), "f"(acc.y));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(C));
+}
+
+__device__ __forceinline__ float sqrt_approx(float x) {
+    float y;
+    asm("sqrt.approx.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float bf16lo(unsigned w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Order-preserving map of an fp32 value onto uint32 (larger float -> larger integer).
+__device__ __forceinline__ unsigned float_key(float z) {
+    unsigned u = __float_as_uint(z);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ void record_status(unsigned long long *st, int code, long long unit) {
+    unsigned long long v = ((unsigned long long)(unsigned)code << 32) | (unsigned long long)(unsigned)unit;
+    atomicCAS(st, 0ull, v);
+}
+
+// Row index (in rows of head_dim elements) of logical slot i of a unit.
+__device__ __forceinline__ long long row_of(const Args &a, int lr, int s, int g, int i) {
+    if (!a.paged) return (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + i;
+    const int page = __ldg(a.block_table + (long long)s * a.max_pages + i / a.page_size);
+    return (((long long)lr * a.n_pages + page) * a.n_kv + g) * (long long)a.page_size + (i % a.page_size);
+}
+
+// k-th (0-based) set bit of m.
+__device__ __forceinline__ int select_bit(unsigned m, int k) {
+    int pos = 0;
+#pragma unroll
+    for (int sh = 16; sh >= 1; sh >>= 1) {
+        const unsigned low = m & ((1u << sh) - 1u);
+        const int c = __popc(low);
+        if (k >= c) {
+            k -= c;
+            m >>= sh;
+            pos += sh;
+        } else {
+            m = low;
+        }
+    }
+    return pos;
+}
+
+// Exclusive scan of n (<= 4 * kThreads) ints in place in shared memory; returns the total.
+// All threads of the block must call it.
+__device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 1 ints */) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    constexpr int PER = 4;
+    int v[PER];
+    int local = 0;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int i = tid * PER + k;
+        v[k] = i < n ? a[i] : 0;
+        local += v[k];
+    }
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+    }
+    if (lane == 31) scratch[warp] = incl;
+    __syncthreads();
+    if (tid == 0) {
+        int run = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const int x = scratch[w];
+            scratch[w] = run;
+            run += x;
+        }
+        scratch[kWarps] = run;
+    }
+    __syncthreads();
+    int ex = scratch[warp] + incl - local;
+#pragma unroll
+    for (int k = 0; k < PER; ++k) {
+        const int i = tid * PER + k;
+        if (i < n) a[i] = ex;
+        ex += v[k];
+    }
+    const int total = scratch[kWarps];
+    __syncthreads();
+    return total;
+}
+
+// Sum of one double per thread over the block; result valid in every thread.
+__device__ double block_sum_f64(double x, double *scratch /* kWarps + 1 */) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    if (lane == 0) scratch[warp] = x;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double r = 0.0;
+        for (int w = 0; w < kWarps; ++w) r += scratch[w];
+        scratch[kWarps] = r;
+    }
+    __syncthreads();
+    const double r = scratch[kWarps];
+    __syncthreads();
+    return r;
+}
+
+// ---------------------------------------------------------------------------------
+// Per-key slice geometry. A key of D dims is split over LPK lanes; each lane holds DH
+// consecutive dims from the first half of the row and the DH dims D/2 further on.
+// ---------------------------------------------------------------------------------
+template <int D, int G>
+struct Geo {
+    static constexpr int DH = (D == 128) ? (G >= 4 ? 4 : (G == 2 ? 8 : 16))
+                                         : (G == 8 ? 2 : (G == 4 ? 4 : (G == 2 ? 8 : 16)));
+    static constexpr int LPK = D / (2 * DH);
+    static constexpr int KPP = 32 / LPK;  // keys per warp per pass
+    static_assert(LPK >= G, "a key needs at least G lanes");
+    static_assert(32 % LPK == 0, "LPK must divide the warp");
+    static_assert(DH % 2 == 0, "DH must be even");
+};
+
+// Load DH consecutive bf16 from smem as DH/2 32-bit words.
+template <int DH>
+__device__ __forceinline__ void load_chunk(const uint16_t *p, unsigned (&w)[DH / 2]) {
+    if constexpr (DH == 2) {
+        w[0] = *reinterpret_cast<const unsigned *>(p);
+    } else if constexpr (DH == 4) {
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        w[0] = x.x; w[1] = x.y;
+    } else if constexpr (DH == 8) {
+        const uint4 x = *reinterpret_cast<const uint4 *>(p);
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+    } else {
+        const uint4 x = *reinterpret_cast<const uint4 *>(p);
+        const uint4 y = *reinterpret_cast<const uint4 *>(p + 8);
+        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
+        w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+    }
+}
+
+// ---------------------------------------------------------------------------------
+// The fused kernel. Grid: (cs * n_units) CTAs in clusters of cs; block: kThreads.
+// ---------------------------------------------------------------------------------
+template <int D, int G, int LAYOUT>
+__global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
+    constexpr int F = D / 2;
+    using GE = Geo<D, G>;
+    constexpr int DH = GE::DH;
+    constexpr int LPK = GE::LPK;
+    constexpr int KPP = GE::KPP;
+    constexpr unsigned FULL = 0xffffffffu;
+
+    extern __shared__ __align__(128) unsigned char smem[];
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cs = a.cs;
+    const int crank = (int)cluster.block_rank();
+    const int unit = blockIdx.x / cs;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const Layout Ly = make_layout(D, G, a.nslot, a.kpc_max, cs);
+
+    float *sc = reinterpret_cast<float *>(smem + Ly.sc);
+    unsigned char *ring = smem + Ly.ring;
+    float *coef_t = reinterpret_cast<float *>(smem + Ly.coef_t);
+    float *coef_w = reinterpret_cast<float *>(smem + Ly.coef_w);
+    double2 *phase = reinterpret_cast<double2 *>(smem + Ly.phase);
+    unsigned *whist = reinterpret_cast<unsigned *>(smem + Ly.whist);
+    unsigned *bhist = reinterpret_cast<unsigned *>(smem + Ly.bhist);
+    int *gh = reinterpret_cast<int *>(smem + Ly.ghist);
+    unsigned *lmask = reinterpret_cast<unsigned *>(smem + Ly.lmask);
+    unsigned *gmask = reinterpret_cast<unsigned *>(smem + Ly.gmask);
+    int *gpre = reinterpret_cast<int *>(smem + Ly.gpre);
+    Xch *xch = reinterpret_cast<Xch *>(smem + Ly.xch);
+    double *dscratch = reinterpret_cast<double *>(smem + Ly.misc);
+    int *iscratch = reinterpret_cast<int *>(smem + Ly.misc + kWarps * 8 * 8);
+    float *bcast = reinterpret_cast<float *>(smem + Ly.misc + kWarps * 8 * 8 + 64 * 4);
+    int *srcidx = reinterpret_cast<int *>(smem + Ly.srcidx);
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Ly.bars);
+
+    const int g = unit % a.n_kv;
+    const int s = (unit / a.n_kv) % a.batch;
+    const int lr = unit / (a.n_kv * a.batch);
+    const int layer = a.layer_begin + lr;
+    const int Hq = a.n_kv * G;
+    const int N = __ldg(a.lens + s);
+    bool talked = false;  // did this cluster use distributed shared memory
+
+    // ---- validation: every CTA of the cluster reaches the same verdict --------------
+    int bad = (N < 0 || N > a.cap_u) ? kDevLenGtCap : 0;
+    if (!bad && a.paged) {
+        const int np = (N + a.page_size - 1) / a.page_size;
+        int mine = 0;
+        for (int p = tid; p < np; p += kThreads) {
+            const int pg = __ldg(a.block_table + (long long)s * a.max_pages + p);
+            if (pg < 0 || pg >= a.n_pages) mine = 1;
+        }
+        if (__syncthreads_or(mine)) bad = kDevBadPage;
+    }
+    if (bad) {
+        if (crank == 0 && tid == 0) {
+            record_status(a.status, bad, unit);
+            if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
+        }
+    }
+    const bool work = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
+
+    if (work) {
+        talked = true;
+        const int kpc = ((N + cs - 1) / cs + 31) / 32 * 32;
+        const int begin = crank * kpc;
+        const int n_local = max(0, min(N - begin, kpc));
+        const int nst = (n_local + kStageRows - 1) / kStageRows;
+        const int nslot = a.nslot;
+        constexpr unsigned kStageBytes = kStageRows * D * 2;
+
+        // ---- start streaming this CTA's keys (TMA bulk copies, per-warp buffers) -----
+        if (lane == 0) {
+            for (int k = 0; k < nslot; ++k) mbar_init(bars + warp * nslot + k, 1);
+            mbar_init_fence();
+        }
+        __syncwarp();
+        auto issue = [&](int st, int slot) {
+            const int row0 = st * kStageRows;
+            const int nrows = min(kStageRows, n_local - row0);
+            const long long r = row_of(a, lr, s, g, begin + row0);
+            uint64_t *bar = bars + warp * nslot + slot;
+            fence_proxy_async_smem();
+            mbar_expect_tx(bar, (unsigned)nrows * D * 2u);
+            tma_load_1d(ring + (size_t)(warp * nslot + slot) * kStageBytes, a.K + r * D,
+                        (unsigned)nrows * D * 2u, bar);
+        };
+        if (lane == 0) {
+            for (int k = 0; k < nslot; ++k) {
+                const int st = warp + k * kWarps;
+                if (st < nst) issue(st, k);
+            }
+        }
+
+        // ---- prologue: per-head coefficients for this sequence's t --------------------
+        const int tq = __ldg(a.t + s);
+        for (int f = tid; f < F; f += kThreads) {
+            double sn, c;
+            sincos(__ldg(a.omega + f) * (double)tq, &sn, &c);
+            phase[f] = make_double2(c, sn);
+        }
+        __syncthreads();
+        for (int idx = tid; idx < G * F; idx += kThreads) {
+            const int h = idx / F, f = idx % F;
+            const long long qi = ((long long)layer * Hq + (long long)g * G + h) * F + f;
+            const double2 q = a.Qc[qi];
+            const double2 e = phase[f];
+            const double re = q.x * e.x - q.y * e.y;
+            const double im = q.x * e.y + q.y * e.x;
+            const int dre = LAYOUT == 0 ? f : 2 * f;
+            const int dim = LAYOUT == 0 ? f + F : 2 * f + 1;
+            coef_t[h * D + dre] = (float)re;
+            coef_t[h * D + dim] = (float)im;
+            coef_w[h * F + f] = __ldg(a.w + qi);
+        }
+        __syncthreads();
+
+        // ---- lane geometry and register-resident coefficients ----------------------
+        const int sub = lane % LPK;
+        const int kw = lane / LPK;
+        int hx = 0;
+        {
+            int cnt = G;
+#pragma unroll
+            for (int m = LPK / 2; m >= 1; m >>= 1) {
+                if (cnt > 1) {
+                    const int half = cnt / 2;
+                    if (lane & m) hx |= half;
+                    cnt = half;
+                }
+            }
+        }
+        float ca[G][DH], cb[G][DH], cw[G][DH];
+#pragma unroll
+        for (int i = 0; i < G; ++i) {
+            const int hq = i ^ hx;
+#pragma unroll
+            for (int j = 0; j < DH; ++j) {
+                ca[i][j] = coef_t[hq * D + sub * DH + j];
+                cb[i][j] = coef_t[hq * D + F + sub * DH + j];
+                if (LAYOUT == 0) {
+                    cw[i][j] = coef_w[hq * F + sub * DH + j];
+                } else {
+                    cw[i][j] = (j < DH / 2) ? coef_w[hq * F + sub * (DH / 2) + j]
+                                            : coef_w[hq * F + D / 4 + sub * (DH / 2) + (j - DH / 2)];
+                }
+            }
+        }
+        const bool writer = (sub & (LPK / G - 1)) == 0;
+        float *raw_row = nullptr;
+        if (a.raw)
+            raw_row = a.raw + (((long long)lr * a.batch + s) * Hq + (long long)g * G + hx) * (long long)a.cap_u + begin;
+
+        // ---- score loop ----------------------------------------------------------------
+        int fail = 0;
+        for (int k = 0;; ++k) {
+            const int st = warp + k * kWarps;
+            if (st >= nst) break;
+            const int slot = k % nslot;
+            const bool landed = __all_sync(FULL, mbar_wait_bounded(bars + warp * nslot + slot,
+                                                                    (unsigned)((k / nslot) & 1)));
+            if (!landed) {
+                // give the copies this warp still has in flight a bounded chance to land
+                // before the buffers are abandoned
+                for (int j = 1; j < nslot; ++j) {
+                    const int kk = k + j;
+                    if (warp + kk * kWarps < nst)
+                        (void)mbar_wait_bounded(bars + warp * nslot + kk % nslot, (unsigned)((kk / nslot) & 1));
+                }
+                fail = 1;
+                break;
+            }
+            const uint16_t *stage =
+                reinterpret_cast<const uint16_t *>(ring + (size_t)(warp * nslot + slot) * kStageBytes);
+#pragma unroll 2
+            for (int pass = 0; pass < kStageRows / KPP; ++pass) {
+                const int r = pass * KPP + kw;
+                const int li = st * kStageRows + r;
+                const uint16_t *row = stage + r * D;
+                unsigned wa[DH / 2], wb[DH / 2];
+                load_chunk<DH>(row + sub * DH, wa);
+                load_chunk<DH>(row + F + sub * DH, wb);
+                float xa[DH], xb[DH];
+#pragma unroll
+                for (int j = 0; j < DH / 2; ++j) {
+                    xa[2 * j] = bf16lo(wa[j]);
+                    xa[2 * j + 1] = bf16hi(wa[j]);
+                    xb[2 * j] = bf16lo(wb[j]);
+                    xb[2 * j + 1] = bf16hi(wb[j]);
+                }
+                float nb[DH];
+                if (LAYOUT == 0) {
+#pragma unroll
+                    for (int j = 0; j < DH; ++j) nb[j] = sqrt_approx(fmaf(xa[j], xa[j], xb[j] * xb[j]));
+                } else {
+#pragma unroll
+                    for (int j = 0; j < DH / 2; ++j) {
+                        nb[j] = sqrt_approx(fmaf(xa[2 * j], xa[2 * j], xa[2 * j + 1] * xa[2 * j + 1]));
+                        nb[DH / 2 + j] = sqrt_approx(fmaf(xb[2 * j], xb[2 * j], xb[2 * j + 1] * xb[2 * j + 1]));
+                    }
+                }
+                float v[G];
+#pragma unroll
+                for (int i = 0; i < G; ++i) {
+                    float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int j = 0; j < DH; j += 2) {
+                        ffma2(acc, make_float2(xa[j], xa[j + 1]), make_float2(ca[i][j], ca[i][j + 1]));
+                        ffma2(acc, make_float2(xb[j], xb[j + 1]), make_float2(cb[i][j], cb[i][j + 1]));
+                        ffma2(acc, make_float2(nb[j], nb[j + 1]), make_float2(cw[i][j], cw[i][j + 1]));
+                    }
+                    v[i] = acc.x + acc.y;
+                }
+                // reduce-scatter over the key's LPK lanes: slot i of a lane holds head i ^ hx,
+                // so partner lanes always exchange the same register indices.
+                {
+                    int cnt = G;
+#pragma unroll
+                    for (int m = LPK / 2; m >= 1; m >>= 1) {
+                        if (cnt > 1) {
+                            const int half = cnt / 2;
+#pragma unroll
+                            for (int i = 0; i < half; ++i) v[i] += __shfl_xor_sync(FULL, v[i + half], m);
+                            cnt = half;
+                        } else {
+                            v[0] += __shfl_xor_sync(FULL, v[0], m);
+                        }
+                    }
+                }
+                if (writer && li < n_local) {
+                    sc[li * G + hx] = v[0];
+                    if (raw_row) raw_row[li] = v[0];
+                }
+            }
+            __syncwarp();
+            const int nxt = st + nslot * kWarps;
+            if (lane == 0 && nxt < nst) issue(nxt, slot);
+        }
+        if (__syncthreads_or(fail)) {
+            if (tid == 0) {
+                record_status(a.status, kDevTimeout, unit);
+                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
+            }
+            fail = 1;
+        }
+
+        // ---- per-head moments over the whole unit (two passes, fp64, cluster-wide) -----
+        {
+            double sum[G];
+            float mn[G], mx[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) { sum[h] = 0.0; mn[h] = __int_as_float(0x7f800000); mx[h] = -mn[h]; }
+            for (int i = tid; i < n_local; i += kThreads) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const float x = sc[i * G + h];
+                    sum[h] += (double)x;
+                    mn[h] = fminf(mn[h], x);
+                    mx[h] = fmaxf(mx[h], x);
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const double t = block_sum_f64(sum[h], dscratch);
+                float lo = mn[h], hi = mx[h];
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+                    lo = fminf(lo, __shfl_xor_sync(FULL, lo, o));
+                    hi = fmaxf(hi, __shfl_xor_sync(FULL, hi, o));
+                }
+                if (lane == 0) { bcast[2 * warp] = lo; bcast[2 * warp + 1] = hi; }
+                __syncthreads();
+                if (tid == 0) {
+                    float l2 = bcast[0], h2 = bcast[1];
+                    for (int w = 1; w < kWarps; ++w) { l2 = fminf(l2, bcast[2 * w]); h2 = fmaxf(h2, bcast[2 * w + 1]); }
+                    xch->sum[h] = t; xch->mn[h] = l2; xch->mx[h] = h2;
+                }
+                __syncthreads();
+            }
+            if (tid == 0) xch->fail = fail;
+        }
+        cluster.sync();
+        // every CTA folds the cluster's partials in rank order: identical mu in every CTA
+        __shared__ double mu_s[8];
+        __shared__ float muf_s[8], inv_s[8];
+        __shared__ int flat_s[8], anyfail_s;
+        if (tid < G) {
+            const int h = tid;
+            double tot = 0.0;
+            float lo = __int_as_float(0x7f800000), hi = -lo;
+            for (int c = 0; c < cs; ++c) {
+                const Xch *r = cluster.map_shared_rank(xch, c);
+                tot += r->sum[h];
+                lo = fminf(lo, r->mn[h]);
+                hi = fmaxf(hi, r->mx[h]);
+            }
+            mu_s[h] = tot / (double)N;
+            flat_s[h] = !(hi > lo);
+        }
+        if (tid == 32) {
+            int f = 0;
+            for (int c = 0; c < cs; ++c) f |= cluster.map_shared_rank(xch, c)->fail;
+            anyfail_s = f;
+        }
+        __syncthreads();
+        {
+            double m2[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) m2[h] = 0.0;
+            for (int i = tid; i < n_local; i += kThreads) {
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    const double dlt = (double)sc[i * G + h] - mu_s[h];
+                    m2[h] += dlt * dlt;
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const double t = block_sum_f64(m2[h], dscratch);
+                if (tid == 0) xch->m2[h] = t;
+            }
+        }
+        cluster.sync();
+        if (tid < G) {
+            const int h = tid;
+            double tot = 0.0;
+            for (int c = 0; c < cs; ++c) tot += cluster.map_shared_rank(xch, c)->m2[h];
+            const double sigma = sqrt(tot / (double)N);
+            muf_s[h] = (float)mu_s[h];
+            inv_s[h] = (flat_s[h] || !(sigma > 0.0)) ? 0.f : (float)(1.0 / sigma);
+        }
+        __syncthreads();
+
+        // ---- z-score, max over the group; the order key replaces the key's first score --
+        float *zrow = a.zmax ? a.zmax + (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + begin
+                             : nullptr;
+        for (int i = tid; i < n_local; i += kThreads) {
+            float z = -__int_as_float(0x7f800000);
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                const float zh = (sc[i * G + h] - muf_s[h]) * inv_s[h];
+                z = fmaxf(z, zh);
+            }
+            z = z + 0.0f;  // -0 -> +0
+            if (zrow) zrow[i] = z;
+            reinterpret_cast<unsigned *>(sc)[i * G] = float_key(z);
+        }
+        __syncthreads();
+        const unsigned *ukey = reinterpret_cast<const unsigned *>(sc);
+
+        if (a.mode == kModePrune && !anyfail_s) {
+            // ---- radix select of the B-th largest key, cluster-wide ------------------------
+            unsigned prefix = 0u, pmask = 0u;
+            int need = a.budget;
+            bool resolved = false;
+            __shared__ int sel_s[3];
+            for (int pass = 0; pass < 4 && !resolved; ++pass) {
+                const int shift = 24 - 8 * pass;
+                unsigned *wh = whist + warp * kBins;
+                for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
+                __syncwarp();
+                const int lim = (n_local + 31) / 32 * 32;
+                for (int i = tid; i < lim; i += kThreads) {
+                    const bool in = i < n_local;
+                    const unsigned u = in ? ukey[i * G] : 0u;
+                    const bool m = in && ((u & pmask) == prefix);
+                    const unsigned bin = (u >> shift) & 255u;
+                    const unsigned act = __ballot_sync(FULL, m);
+                    if (m) {
+                        const unsigned peers = __match_any_sync(act, bin);
+                        if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
+                    }
+                }
+                __syncthreads();
+                unsigned *bh = bhist + (pass & 1) * kBins;
+                for (int b = tid; b < kBins; b += kThreads) {
+                    unsigned c = 0u;
+                    for (int w = 0; w < kWarps; ++w) c += whist[w * kBins + b];
+                    bh[b] = c;
+                }
+                cluster.sync();
+                // global histogram, bins reversed so that index 0 is the top bin; every CTA
+                // folds the cluster's histograms in the same order and finds the same bin
+                for (int b = tid; b < kBins; b += kThreads) {
+                    unsigned c = 0u;
+                    for (int r = 0; r < cs; ++r) c += cluster.map_shared_rank(bh, r)[b];
+                    gh[kBins - 1 - b] = (int)c;  // reversed: index 0 is the top bin
+                }
+                __syncthreads();
+                // inclusive scan over reversed bins
+                if (warp == 0) {
+                    int run = 0;
+                    for (int base = 0; base < kBins; base += 32) {
+                        int x = gh[base + lane];
+                        int incl = x;
+#pragma unroll
+                        for (int o = 1; o < 32; o <<= 1) {
+                            const int y = __shfl_up_sync(FULL, incl, o);
+                            if (lane >= o) incl += y;
+                        }
+                        incl += run;
+                        const int above = incl - x;
+                        if (above < need && incl >= need) {
+                            sel_s[0] = kBins - 1 - (base + lane);
+                            sel_s[1] = above;
+                            sel_s[2] = x;
+                        }
+                        run = __shfl_sync(FULL, incl, 31);
+                    }
+                }
+                __syncthreads();
+                const int bstar = sel_s[0];
+                need -= sel_s[1];
+                const int cnt = sel_s[2];
+                prefix |= (unsigned)bstar << shift;
+                pmask |= 255u << shift;
+                resolved = (cnt == need);
+                __syncthreads();
+            }
+            const bool tie = !resolved;
+
+            // ---- keep mask: word per 32 local keys; exact ties ranked by slot -------------
+            const int nwl = kpc / 32;
+            int *tw = gpre;  // scratch for per-word tie counts before gpre is built
+            int tie_off = 0;
+            if (tie) {
+                for (int wi = warp; wi < nwl; wi += kWarps) {
+                    const int i = wi * 32 + lane;
+                    const bool eq = i < n_local && ukey[i * G] == prefix;
+                    const unsigned bb = __ballot_sync(FULL, eq);
+                    if (lane == 0) tw[wi] = __popc(bb);
+                }
+                __syncthreads();
+                const int my_ties = block_exclusive_scan(tw, nwl, iscratch);
+                if (tid == 0) xch->ties = my_ties;
+                cluster.sync();
+                if (tid == 0) {
+                    int off = 0;
+                    for (int c = 0; c < crank; ++c) off += cluster.map_shared_rank(xch, c)->ties;
+                    iscratch[kWarps + 1] = off;
+                }
+                __syncthreads();
+                tie_off = iscratch[kWarps + 1];
+            }
+            for (int wi = warp; wi < nwl; wi += kWarps) {
+                const int i = wi * 32 + lane;
+                const bool in = i < n_local;
+                const unsigned u = in ? ukey[i * G] : 0u;
+                const bool gt = in && (u & pmask) > prefix;
+                const bool eq = in && (u & pmask) == prefix;
+                bool keep = gt || (eq && !tie);
+                if (tie) {
+                    const unsigned eb = __ballot_sync(FULL, eq);
+                    const int rank = tie_off + tw[wi] + __popc(eb & ((1u << lane) - 1u));
+                    keep = gt || (eq && rank < need);
+                }
+                const unsigned kb = __ballot_sync(FULL, keep);
+                if (lane == 0) lmask[wi] = kb;
+            }
+            cluster.sync();
+            // global mask and its word prefix (identical in all CTAs)
+            const int nwt = cs * nwl;
+            for (int wg = tid; wg < nwt; wg += kThreads) {
+                const int c = wg / nwl, wi = wg % nwl;
+                const unsigned m = cluster.map_shared_rank(lmask, c)[wi];
+                gmask[wg] = m;
+                gpre[wg] = __popc(m);
+            }
+            __syncthreads();
+            // nwt can exceed 4 * kThreads for tiny kpc * large cs only when nwt > 1024;
+            // the host keeps cs * kpc <= 32768 * 4 so nwt <= 4096 -> scan in 4 chunks
+            {
+                int run = 0;
+                for (int base = 0; base < nwt; base += 4 * kThreads) {
+                    const int n = min(4 * kThreads, nwt - base);
+                    const int tot = block_exclusive_scan(gpre + base, n, iscratch);
+                    for (int q = tid; q < n; q += kThreads) gpre[base + q] += run;
+                    __syncthreads();
+                    run += tot;
+                }
+                if (tid == 0) gpre[nwt] = run;
+                __syncthreads();
+            }
+            const int M = a.budget;
+            // the mask must hold exactly M keys; anything else is an internal error and the
+            // unit is left untouched rather than copied from a wrong index
+            const bool count_ok = gpre[nwt] == M;
+            if (!count_ok && crank == 0 && tid == 0) {
+                record_status(a.status, kDevInternal, unit);
+                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
+            }
+
+            // ---- in-place stable compaction in ascending destination rounds ---------------
+            const int S = Ly.stage_rows;
+            uint16_t *stK = reinterpret_cast<uint16_t *>(smem);  // region A
+            uint16_t *stV = stK + (size_t)S * D;
+            int32_t *stP = reinterpret_cast<int32_t *>(stV + (size_t)S * D);
+            constexpr int LPR = D / 8;  // lanes per row (16 bytes each)
+            constexpr int RPW = 32 / LPR;
+            const int R = S * cs;
+            for (int base = 0; count_ok && base < M; base += R) {
+                const int d0 = base + crank * S;
+                const int nd = max(0, min(M - d0, S));
+                for (int j = tid; j < nd; j += kThreads) {
+                    const int dst = d0 + j;
+                    int lo = 0, hi = nwt;  // largest w with gpre[w] <= dst
+                    while (hi - lo > 1) {
+                        const int mid = (lo + hi) >> 1;
+                        if (gpre[mid] <= dst) lo = mid; else hi = mid;
+                    }
+                    const int w = lo;
+                    const int bit = select_bit(gmask[w], dst - gpre[w]);
+                    const int c = w / nwl;
+                    srcidx[j] = min(c * kpc + (w % nwl) * 32 + bit, N - 1);
+                }
+                __syncthreads();
+                for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
+                    const long long srow = row_of(a, lr, s, g, srcidx[rr]);
+                    const int q = lane % LPR;
+                    cp_async16(stK + (size_t)rr * D + q * 8, a.K + srow * D + q * 8);
+                    cp_async16(stV + (size_t)rr * D + q * 8, a.V + srow * D + q * 8);
+                    if (q == 0) cp_async4(stP + rr, a.pos + srow);
+                }
+                cp_async_wait_all();
+                __syncthreads();
+                cluster.sync();  // every source row of this round is now in shared memory
+                for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
+                    const long long drow = row_of(a, lr, s, g, d0 + rr);
+                    const int q = lane % LPR;
+                    const uint4 xk = *reinterpret_cast<const uint4 *>(stK + (size_t)rr * D + q * 8);
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(stV + (size_t)rr * D + q * 8);
+                    *reinterpret_cast<uint4 *>(a.K + drow * D + q * 8) = xk;
+                    *reinterpret_cast<uint4 *>(a.V + drow * D + q * 8) = xv;
+                    if (q == 0) a.pos[drow] = stP[rr];
+                }
+                __syncthreads();
+            }
+        } else if (a.mode == kModePrune && anyfail_s) {
+            if (crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
+        }
+    }
+
+    // nobody leaves while a peer may still read its shared memory
+    if (talked) cluster.sync();
+
+    // ---- the last CTA to finish publishes the new lengths ------------------------------
+    if (a.mode == kModePrune && a.lens_out) {
+        __shared__ int last_s;
+        __syncthreads();
+        if (tid == 0) {
+            __threadfence();
+            const unsigned tk = atomicAdd(a.counter, 1u);
+            last_s = (tk == gridDim.x - 1);
+        }
+        __syncthreads();
+        if (last_s) {
+            __threadfence();
+            for (int q = tid; q < a.batch; q += kThreads) {
+                const int n = a.lens[q];
+                const int refused = a.seq_bad ? atomicExch(a.seq_bad + q, 0) : 0;
+                a.lens_out[q] = refused ? n : min(n, a.budget);
+            }
+            __syncthreads();
+            if (tid == 0) atomicExch(a.counter, 0u);
+        }
+    }
+}
+
+}  // namespace tri

@@ -199,6 +199,20 @@ class Cache:
     def paged(self) -> bool:
         return self.block_table is not None
 
+    def to(self, device) -> "Cache":
+        """Move every tensor of the cache to ``device`` (in place); returns self."""
+        self.K, self.V, self.pos = self.K.to(device), self.V.to(device), self.pos.to(device)
+        self.lens, self.t = self.lens.to(device), self.t.to(device)
+        if self.block_table is not None:
+            self.block_table = self.block_table.to(device)
+        return self
+
+    def clone(self) -> "Cache":
+        c = Cache(self.spec, self.K.clone(), self.V.clone(), self.pos.clone(), self.lens.clone(),
+                  self.t.clone(), None if self.block_table is None else self.block_table.clone(),
+                  self.n_pages, self.cap, (self.q_mean, self.q_norm_mean, self.R, self.offsets))
+        return c
+
     @property
     def n_units(self) -> int:
         s = self.spec
