@@ -268,6 +268,7 @@ def run_ours(args, rank, world, dist_mod):
         "clocks": clk.summary(),
         "gpu_launches": args.steps,
         "keys_per_rank": keys_rank,
+        "lens": lens_host,
     }
 
     # ---- end to end through the public API with host buffers ----------------------------
@@ -480,7 +481,7 @@ def main():
         "data": "synthetic",
         "config": {"workload": args.workload, "layers": spec.n_layers, "kv_heads": spec.n_kv_heads,
                    "group": spec.group, "head_dim": spec.head_dim, "batch_per_gpu": spec.batch,
-                   "keys_per_unit": list(sorted(set(int(x) for x in cache.lens_host)))[:4],
+                   "keys_per_unit": sorted(set(int(x) for x in res["lens"]))[:4],
                    "budget": spec.budget, "parallelism": f"replicas x{world} (sequence shards, no collective)",
                    "l2": "256 MiB buffer written between steps; 19 GB of inputs > L2",
                    "timed": "CUDA events around the tri_prune launch; row restore between steps untimed"},
