@@ -47,7 +47,7 @@ namespace cg = cooperative_groups;
 
 constexpr int kStageRows = 16;      // rows per TMA bulk copy (one copy never crosses a page)
 constexpr int kBins = 256;          // radix digit width: 8 bits
-constexpr int kWarps = 8;           // warps per CTA
+constexpr int kWarps = 12;          // warps per CTA
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxCluster = 16;
 constexpr int kModePrune = 0;
@@ -334,36 +334,60 @@ __device__ double block_sum_f64(double x, double *scratch /* kWarps + 1 */) {
 
 // ---------------------------------------------------------------------------------
 // Per-key slice geometry. A key of D dims is split over LPK lanes; each lane holds DH
-// consecutive dims from the first half of the row and the DH dims D/2 further on.
+// consecutive dims from the first half of the row and the DH dims D/2 further on, i.e.
+// DH whole bands in either rotary layout. DH is chosen so that a lane keeps 3 * DH * G
+// (= 96) coefficients in registers: its DH trig coefficients of each half and its DH
+// norm weights, for every head of the group.
 // ---------------------------------------------------------------------------------
 template <int D, int G>
 struct Geo {
-    static constexpr int DH = (D == 128) ? (G >= 4 ? 4 : (G == 2 ? 8 : 16))
-                                         : (G == 8 ? 2 : (G == 4 ? 4 : (G == 2 ? 8 : 16)));
+    static constexpr int DH_REG = G == 8 ? 4 : (G == 4 ? 8 : (G == 2 ? 16 : 32));
+    static constexpr int DH = DH_REG < D / 4 ? DH_REG : D / 4;  // at least 2 lanes per key
     static constexpr int LPK = D / (2 * DH);
     static constexpr int KPP = 32 / LPK;  // keys per warp per pass
+    static constexpr int NP = DH / 2;     // float2 pairs per half-chunk
     static_assert(LPK >= G, "a key needs at least G lanes");
-    static_assert(32 % LPK == 0, "LPK must divide the warp");
-    static_assert(DH % 2 == 0, "DH must be even");
+    static_assert(LPK >= 2 && 32 % LPK == 0, "LPK must divide the warp");
+    static_assert(KPP <= kStageRows, "a pass must fit in one stage");
+    static_assert(DH % 4 == 0, "DH must be a multiple of 4");
 };
 
 // Load DH consecutive bf16 from smem as DH/2 32-bit words.
 template <int DH>
 __device__ __forceinline__ void load_chunk(const uint16_t *p, unsigned (&w)[DH / 2]) {
-    if constexpr (DH == 2) {
-        w[0] = *reinterpret_cast<const unsigned *>(p);
-    } else if constexpr (DH == 4) {
+    if constexpr (DH == 4) {
         const uint2 x = *reinterpret_cast<const uint2 *>(p);
         w[0] = x.x; w[1] = x.y;
-    } else if constexpr (DH == 8) {
-        const uint4 x = *reinterpret_cast<const uint4 *>(p);
-        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
     } else {
-        const uint4 x = *reinterpret_cast<const uint4 *>(p);
-        const uint4 y = *reinterpret_cast<const uint4 *>(p + 8);
-        w[0] = x.x; w[1] = x.y; w[2] = x.z; w[3] = x.w;
-        w[4] = y.x; w[5] = y.y; w[6] = y.z; w[7] = y.w;
+#pragma unroll
+        for (int q = 0; q < DH / 8; ++q) {
+            const uint4 x = *reinterpret_cast<const uint4 *>(p + 8 * q);
+            w[4 * q] = x.x; w[4 * q + 1] = x.y; w[4 * q + 2] = x.z; w[4 * q + 3] = x.w;
+        }
     }
+}
+
+// bf16 pairs -> fp32 pairs. Half layout: pair p = dims (2p, 2p+1). Interleaved layout:
+// pair 2i = dims (4i, 4i+2), pair 2i+1 = dims (4i+1, 4i+3), so that the two members of
+// each rotary band land in matching lanes of two pairs (one fp32x2 square-sum per two bands).
+template <int NP, int LAYOUT>
+__device__ __forceinline__ void unpack_pairs(const unsigned (&w)[NP], float2 (&x)[NP]) {
+    if constexpr (LAYOUT == 0) {
+#pragma unroll
+        for (int p = 0; p < NP; ++p) x[p] = make_float2(bf16lo(w[p]), bf16hi(w[p]));
+    } else {
+#pragma unroll
+        for (int i = 0; i < NP / 2; ++i) {
+            x[2 * i] = make_float2(bf16lo(w[2 * i]), bf16lo(w[2 * i + 1]));
+            x[2 * i + 1] = make_float2(bf16hi(w[2 * i]), bf16hi(w[2 * i + 1]));
+        }
+    }
+}
+
+// Dim index (within the lane's DH-dim chunk) of element e (0 = .x, 1 = .y) of pair p.
+template <int LAYOUT>
+__host__ __device__ constexpr int pair_dim(int p, int e) {
+    return LAYOUT == 0 ? 2 * p + e : 4 * (p / 2) + (p % 2) + 2 * e;
 }
 
 // ---------------------------------------------------------------------------------
@@ -501,20 +525,30 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                 }
             }
         }
-        float ca[G][DH], cb[G][DH], cw[G][DH];
+        constexpr int NP = GE::NP;
+        // register-resident coefficients, in the pair order the unpack produces
+        float2 ca[G][NP], cb[G][NP], cw[G][NP];
 #pragma unroll
         for (int i = 0; i < G; ++i) {
             const int hq = i ^ hx;
 #pragma unroll
-            for (int j = 0; j < DH; ++j) {
-                ca[i][j] = coef_t[hq * D + sub * DH + j];
-                cb[i][j] = coef_t[hq * D + F + sub * DH + j];
+            for (int p = 0; p < NP; ++p) {
+                const int d0 = pair_dim<LAYOUT>(p, 0), d1 = pair_dim<LAYOUT>(p, 1);
+                ca[i][p] = make_float2(coef_t[hq * D + sub * DH + d0], coef_t[hq * D + sub * DH + d1]);
+                cb[i][p] = make_float2(coef_t[hq * D + F + sub * DH + d0], coef_t[hq * D + F + sub * DH + d1]);
+                // norm pairs: half layout -> bands (sub*DH + 2p, +1); interleaved -> pairs
+                // 0..NP/2-1 come from the first-half chunk, the rest from the second
+                int b0, b1;
                 if (LAYOUT == 0) {
-                    cw[i][j] = coef_w[hq * F + sub * DH + j];
+                    b0 = sub * DH + 2 * p;
+                    b1 = b0 + 1;
                 } else {
-                    cw[i][j] = (j < DH / 2) ? coef_w[hq * F + sub * (DH / 2) + j]
-                                            : coef_w[hq * F + D / 4 + sub * (DH / 2) + (j - DH / 2)];
+                    const int base = (p < NP / 2) ? sub * (DH / 2) : D / 4 + sub * (DH / 2);
+                    const int q = (p < NP / 2) ? p : p - NP / 2;
+                    b0 = base + 2 * q;
+                    b1 = b0 + 1;
                 }
+                cw[i][p] = make_float2(coef_w[hq * F + b0], coef_w[hq * F + b1]);
             }
         }
         const bool writer = (sub & (LPK / G - 1)) == 0;
@@ -551,34 +585,35 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                 unsigned wa[DH / 2], wb[DH / 2];
                 load_chunk<DH>(row + sub * DH, wa);
                 load_chunk<DH>(row + F + sub * DH, wb);
-                float xa[DH], xb[DH];
-#pragma unroll
-                for (int j = 0; j < DH / 2; ++j) {
-                    xa[2 * j] = bf16lo(wa[j]);
-                    xa[2 * j + 1] = bf16hi(wa[j]);
-                    xb[2 * j] = bf16lo(wb[j]);
-                    xb[2 * j + 1] = bf16hi(wb[j]);
-                }
-                float nb[DH];
+                float2 xa[NP], xb[NP], nb[NP];
+                unpack_pairs<NP, LAYOUT>(wa, xa);
+                unpack_pairs<NP, LAYOUT>(wb, xb);
                 if (LAYOUT == 0) {
 #pragma unroll
-                    for (int j = 0; j < DH; ++j) nb[j] = sqrt_approx(fmaf(xa[j], xa[j], xb[j] * xb[j]));
+                    for (int p = 0; p < NP; ++p) {
+                        const float2 q2 = __ffma2_rn(xb[p], xb[p], __fmul2_rn(xa[p], xa[p]));
+                        nb[p] = make_float2(sqrt_approx(q2.x), sqrt_approx(q2.y));
+                    }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < DH / 2; ++j) {
-                        nb[j] = sqrt_approx(fmaf(xa[2 * j], xa[2 * j], xa[2 * j + 1] * xa[2 * j + 1]));
-                        nb[DH / 2 + j] = sqrt_approx(fmaf(xb[2 * j], xb[2 * j], xb[2 * j + 1] * xb[2 * j + 1]));
+                    for (int i = 0; i < NP / 2; ++i) {
+                        const float2 qa = __ffma2_rn(xa[2 * i + 1], xa[2 * i + 1], __fmul2_rn(xa[2 * i], xa[2 * i]));
+                        const float2 qb = __ffma2_rn(xb[2 * i + 1], xb[2 * i + 1], __fmul2_rn(xb[2 * i], xb[2 * i]));
+                        nb[i] = make_float2(sqrt_approx(qa.x), sqrt_approx(qa.y));
+                        nb[NP / 2 + i] = make_float2(sqrt_approx(qb.x), sqrt_approx(qb.y));
                     }
                 }
                 float v[G];
 #pragma unroll
                 for (int i = 0; i < G; ++i) {
-                    float2 acc = make_float2(0.f, 0.f);
+                    float2 acc = __fmul2_rn(xa[0], ca[i][0]);
+                    acc = __ffma2_rn(xb[0], cb[i][0], acc);
+                    acc = __ffma2_rn(nb[0], cw[i][0], acc);
 #pragma unroll
-                    for (int j = 0; j < DH; j += 2) {
-                        ffma2(acc, make_float2(xa[j], xa[j + 1]), make_float2(ca[i][j], ca[i][j + 1]));
-                        ffma2(acc, make_float2(xb[j], xb[j + 1]), make_float2(cb[i][j], cb[i][j + 1]));
-                        ffma2(acc, make_float2(nb[j], nb[j + 1]), make_float2(cw[i][j], cw[i][j + 1]));
+                    for (int p = 1; p < NP; ++p) {
+                        acc = __ffma2_rn(xa[p], ca[i][p], acc);
+                        acc = __ffma2_rn(xb[p], cb[i][p], acc);
+                        acc = __ffma2_rn(nb[p], cw[i][p], acc);
                     }
                     v[i] = acc.x + acc.y;
                 }
@@ -651,26 +686,38 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             if (tid == 0) xch->fail = fail;
         }
         cluster.sync();
-        // every CTA folds the cluster's partials in rank order: identical mu in every CTA
+        // every CTA gathers the cluster's partials (one remote load per thread, all in
+        // flight together) and folds them in rank order: identical mu in every CTA
+        __shared__ double part_d[kMaxCluster][8];
+        __shared__ float part_lo[kMaxCluster][8], part_hi[kMaxCluster][8];
+        __shared__ int part_fail[kMaxCluster];
         __shared__ double mu_s[8];
         __shared__ float muf_s[8], inv_s[8];
         __shared__ int flat_s[8], anyfail_s;
+        for (int idx = tid; idx < cs * G; idx += kThreads) {
+            const int c = idx / G, h = idx % G;
+            const Xch *r = cluster.map_shared_rank(xch, c);
+            part_d[c][h] = r->sum[h];
+            part_lo[c][h] = r->mn[h];
+            part_hi[c][h] = r->mx[h];
+            if (h == 0) part_fail[c] = r->fail;
+        }
+        __syncthreads();
         if (tid < G) {
             const int h = tid;
             double tot = 0.0;
             float lo = __int_as_float(0x7f800000), hi = -lo;
             for (int c = 0; c < cs; ++c) {
-                const Xch *r = cluster.map_shared_rank(xch, c);
-                tot += r->sum[h];
-                lo = fminf(lo, r->mn[h]);
-                hi = fmaxf(hi, r->mx[h]);
+                tot += part_d[c][h];
+                lo = fminf(lo, part_lo[c][h]);
+                hi = fmaxf(hi, part_hi[c][h]);
             }
             mu_s[h] = tot / (double)N;
             flat_s[h] = !(hi > lo);
         }
         if (tid == 32) {
             int f = 0;
-            for (int c = 0; c < cs; ++c) f |= cluster.map_shared_rank(xch, c)->fail;
+            for (int c = 0; c < cs; ++c) f |= part_fail[c];
             anyfail_s = f;
         }
         __syncthreads();
@@ -692,10 +739,15 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             }
         }
         cluster.sync();
+        for (int idx = tid; idx < cs * G; idx += kThreads) {
+            const int c = idx / G, h = idx % G;
+            part_d[c][h] = cluster.map_shared_rank(xch, c)->m2[h];
+        }
+        __syncthreads();
         if (tid < G) {
             const int h = tid;
             double tot = 0.0;
-            for (int c = 0; c < cs; ++c) tot += cluster.map_shared_rank(xch, c)->m2[h];
+            for (int c = 0; c < cs; ++c) tot += part_d[c][h];
             const double sigma = sqrt(tot / (double)N);
             muf_s[h] = (float)mu_s[h];
             inv_s[h] = (flat_s[h] || !(sigma > 0.0)) ? 0.f : (float)(1.0 / sigma);
@@ -753,8 +805,13 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                 // global histogram, bins reversed so that index 0 is the top bin; every CTA
                 // folds the cluster's histograms in the same order and finds the same bin
                 for (int b = tid; b < kBins; b += kThreads) {
+                    unsigned part[kMaxCluster];
+#pragma unroll
+                    for (int r = 0; r < kMaxCluster; ++r)
+                        part[r] = r < cs ? cluster.map_shared_rank(bh, r)[b] : 0u;
                     unsigned c = 0u;
-                    for (int r = 0; r < cs; ++r) c += cluster.map_shared_rank(bh, r)[b];
+#pragma unroll
+                    for (int r = 0; r < kMaxCluster; ++r) c += part[r];
                     gh[kBins - 1 - b] = (int)c;  // reversed: index 0 is the top bin
                 }
                 __syncthreads();
