@@ -35,6 +35,8 @@ struct tri_ctx {
     unsigned int *d_counter = nullptr;
     int32_t *d_seq_bad = nullptr;
     int seq_bad_cap = 0;
+    float *d_scratch = nullptr;      // per-cluster score slots of the persistent grid
+    size_t scratch_bytes = 0;
     // tuning (0 = automatic)
     int tune_cs = 0;
     int tune_nslot = 0;
@@ -101,9 +103,13 @@ tri_status cuda_fail(tri_ctx *c, cudaError_t e, const char *what, tri_status st 
 }
 
 struct Plan {
-    int cs = 0, nslot = 0, kpc = 0;
+    int cs = 0, nslot = 0, kpc = 0, n_clusters = 0;
     size_t smem = 0;
 };
+
+// Live score slots should stay well inside the 126 MB L2 so that the scores written during
+// streaming are read back from L2.
+constexpr double kScoreL2Budget = 100.0 * 1024 * 1024;
 
 std::mutex g_attr_mu;
 
@@ -125,50 +131,69 @@ cudaError_t prepare_kernel(KernelFn fn, int max_optin) {
     return cudaSuccess;
 }
 
-// Pick the cluster size: the smallest that fits the unit's scores on chip and still gives
-// the GPU at least two CTAs per SM to schedule, else the largest that fits.
+// Clusters that can be resident at once for this shape (0 if it cannot launch).
+int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem) {
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)cs);
+    cfg.blockDim = dim3(tri::kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    const cudaError_t e = cudaOccupancyMaxActiveClusters(&n, fn, &cfg);
+    if (e != cudaSuccess) {
+        cuda_fail(c, e, "cudaOccupancyMaxActiveClusters");
+        return 0;
+    }
+    return n;
+}
+
+// Pick the launch shape of the persistent grid. A cluster of cs CTAs shares one unit; the
+// grid holds as many clusters as can be resident (two CTAs per SM). cs is the smallest
+// power of two that (a) gives every resident CTA slot a unit to work on and (b) keeps the
+// live score slots (one per resident cluster) within the L2 budget; if none does both,
+// the largest cs that fits.
 tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Plan *out) {
     cudaFuncAttributes fa;
     cudaError_t fe = cudaFuncGetAttributes(&fa, fn);
     if (fe != cudaSuccess) return cuda_fail(c, fe, "cudaFuncGetAttributes");
     const size_t budget = (size_t)c->max_smem_optin - fa.sharedSizeBytes;
-    const int nslot = c->tune_nslot > 0 ? c->tune_nslot : 2;
+    const double unit_bytes = (double)cap_u * c->G * 4.0;  // scores; order keys usually stay on chip
     Plan best;
     for (int cs = 1; cs <= tri::kMaxCluster; cs *= 2) {
         if (c->tune_cs > 0 && cs != c->tune_cs) continue;
         const long long kpc = ((long long)(cap_u + cs - 1) / cs + 31) / 32 * 32;
-        if (kpc > 32768) continue;
-        const tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
-        if (Ly.total > budget || Ly.stage_rows < 16) continue;
-        // the cluster must be schedulable with this much shared memory per CTA
-        {
-            cudaLaunchConfig_t cfg;
-            std::memset(&cfg, 0, sizeof cfg);
-            cfg.gridDim = dim3((unsigned)cs);
-            cfg.blockDim = dim3(tri::kThreads);
-            cfg.dynamicSmemBytes = Ly.total;
-            cudaLaunchAttribute attr[1];
-            attr[0].id = cudaLaunchAttributeClusterDimension;
-            attr[0].val.clusterDim.x = (unsigned)cs;
-            attr[0].val.clusterDim.y = 1;
-            attr[0].val.clusterDim.z = 1;
-            cfg.attrs = attr;
-            cfg.numAttrs = 1;
-            int nclusters = 0;
-            const cudaError_t oe = cudaOccupancyMaxActiveClusters(&nclusters, fn, &cfg);
-            if (oe != cudaSuccess) {
-                cuda_fail(c, oe, "cudaOccupancyMaxActiveClusters");
-                continue;
+        if (kpc * cs / 32 > 16384) continue;  // global keep mask must fit on chip
+        int nslot = c->tune_nslot > 0 ? c->tune_nslot : 3;
+        tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
+        int res = 0;
+        while (nslot >= 1) {
+            Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
+            if (Ly.total <= budget && Ly.stage_rows >= 16) {
+                res = resident_clusters(c, fn, cs, Ly.total);
+                if (res >= 1 && (c->tune_nslot > 0 || res * cs >= 2 * c->sm_count || nslot == 1)) break;
+                if (res >= 1 && c->tune_nslot > 0) break;
             }
-            if (nclusters < 1) continue;
+            if (c->tune_nslot > 0) { res = 0; break; }
+            --nslot;
         }
+        if (res < 1 || nslot < 1) continue;
         Plan p;
         p.cs = cs;
         p.nslot = nslot;
         p.kpc = (int)kpc;
         p.smem = Ly.total;
+        p.n_clusters = (int)std::min<long long>(n_units, res);
         best = p;
-        if (n_units * cs >= 2LL * c->sm_count) break;
+        const bool fills = n_units * cs >= (long long)res * cs;  // every resident cluster has a unit
+        const bool fits_l2 = (double)p.n_clusters * unit_bytes <= kScoreL2Budget;
+        if (fills && fits_l2) break;
     }
     if (best.cs == 0) return TRI_EUNSUPPORTED;
     *out = best;
@@ -221,6 +246,17 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     tri_status st = plan_launch(c, fn, (int)cap_u, n_units, &plan);
     if (st != TRI_OK) return st;
 
+    const long long slot_floats = ((long long)cap_u * (c->G + 1) + 31) / 32 * 32;
+    const size_t need = (size_t)slot_floats * 4 * plan.n_clusters;
+    if (need > c->scratch_bytes) {
+        cudaFree(c->d_scratch);  // synchronises the device: no call still uses the old slots
+        c->d_scratch = nullptr;
+        c->scratch_bytes = 0;
+        ce = cudaMalloc(&c->d_scratch, need);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaMalloc(scratch)", TRI_ENOMEM);
+        c->scratch_bytes = need;
+    }
+
     const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
     if (finalize && kv->batch > c->seq_bad_cap) {
         cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
@@ -258,13 +294,16 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     a.cs = plan.cs;
     a.kpc_max = plan.kpc;
     a.nslot = plan.nslot;
+    a.n_units = (int)n_units;
+    a.scratch = c->d_scratch;
+    a.slot_floats = slot_floats;
     a.status = c->d_status;
     a.counter = c->d_counter;
     a.seq_bad = finalize ? c->d_seq_bad : nullptr;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3((unsigned)(n_units * plan.cs));
+    cfg.gridDim = dim3((unsigned)(plan.n_clusters * plan.cs));
     cfg.blockDim = dim3(tri::kThreads);
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
@@ -323,6 +362,7 @@ tri_status tri_destroy(tri_ctx *c) {
     cudaFree(c->d_status);
     cudaFree(c->d_counter);
     cudaFree(c->d_seq_bad);
+    cudaFree(c->d_scratch);
     delete c;
     return TRI_OK;
 }

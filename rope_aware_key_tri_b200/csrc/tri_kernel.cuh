@@ -6,8 +6,9 @@
 //   [10100]      the 10100.com article 127765992 on TriAttention
 //   [Summary]    "TriAttention：面向长文本推理的高效KV缓存压缩，2.5倍吞吐提升与10.7倍内存缩减"
 //
-// One thread-block cluster owns one unit (sequence s, layer l, KV head g) and runs the
-// whole pass on it without a round trip through HBM:
+// A persistent grid of thread-block clusters (two CTAs per SM) walks the units; one
+// cluster of cs CTAs owns one unit (sequence s, layer l, KV head g) at a time and runs
+// the whole pass on it:
 //
 //   prologue  C_{h,f} = (qbar_{h,f} A_f) e^{i omega_f t}, with A_f = mean_delta e^{i omega_f delta}
 //             (fp64 phase, rounded to fp32 once). Because the stored key is post-RoPE,
@@ -17,11 +18,12 @@
 //             becomes one dot product per key and head; positions drop out.
 //   score     per key: s_h = sum_j c_{h,j} k~_j + sum_f w_{h,f} |k~_f|, w = (1 - R) E|q|
 //             ([Stage] item 2 with the (1 - R) weight of [10100] §TriAttention方法). Keys
-//             stream from HBM by TMA bulk copies (cp.async.bulk, mbarrier completion)
-//             into per-warp double buffers; each key is split over LPK lanes, every lane
-//             keeps its slice of the coefficients in registers and accumulates with
-//             packed fp32x2 FMAs; a reduce-scatter over the lanes finishes the G heads.
-//             Scores stay in shared memory.
+//             stream from HBM by TMA bulk copies (cp.async.bulk, mbarrier completion,
+//             evict-first L2 hint) into per-warp buffers; each key is split over LPK lanes,
+//             every lane keeps its slice of the coefficients in registers and accumulates
+//             with packed fp32x2 FMAs; a reduce-scatter over the lanes finishes the G heads.
+//             Scores go to a per-cluster scratch slot with an evict-last L2 hint, so they
+//             are re-read from L2, not HBM.
 //   z / max   per head: mean and population std over all of the unit's keys (fp64 sums
 //             exchanged between the cluster's CTAs through distributed shared memory),
 //             z = (s - mu) / sigma (0 for a flat head), max over the G heads
@@ -47,8 +49,9 @@ namespace cg = cooperative_groups;
 
 constexpr int kStageRows = 16;      // rows per TMA bulk copy (one copy never crosses a page)
 constexpr int kBins = 256;          // radix digit width: 8 bits
-constexpr int kWarps = 12;          // warps per CTA
+constexpr int kWarps = 6;           // warps per CTA (two CTAs per SM)
 constexpr int kThreads = kWarps * 32;
+constexpr int kMinBlocks = 2;
 constexpr int kMaxCluster = 16;
 constexpr int kModePrune = 0;
 constexpr int kModeScore = 1;
@@ -56,7 +59,8 @@ constexpr int kDevLenGtCap = 1;
 constexpr int kDevBadPage = 2;
 constexpr int kDevTimeout = 3;
 constexpr int kDevInternal = 4;
-constexpr long long kWaitLimit = 1ll << 22;   // bounded mbarrier polls (with backoff: ~1 s)
+constexpr int kWaitTries = 1024;             // bounded mbarrier waits ...
+constexpr unsigned kWaitSuspendNs = 1000000; // ... each suspending the warp for up to 1 ms
 
 struct Args {
     uint16_t *K;                 // bf16 bits
@@ -70,6 +74,7 @@ struct Args {
     int paged, page_size, max_pages, n_pages;
     int layer_begin;
     int budget;
+    int n_units;
     const double *omega;         // [F]
     const double2 *Qc;           // [L][Hq][F]  qbar * A
     const float *w;              // [L][Hq][F]  (1 - R) E|q|
@@ -79,6 +84,8 @@ struct Args {
     int cs;                      // cluster size (CTAs per unit)
     int kpc_max;                 // key capacity of one CTA (multiple of 32)
     int nslot;                   // TMA buffers per warp
+    float *scratch;              // per-cluster slots: [cap_u][G] scores then [cap_u] order keys
+    long long slot_floats;       // floats per slot
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
     int32_t *seq_bad;            // [batch] sequences the device refused this call
@@ -97,10 +104,9 @@ struct Xch {
 };
 
 struct Layout {
-    unsigned sc, ring, coef_t, coef_w, phase, whist, bhist, ghist, lmask, gmask, gpre, xch, misc,
+    unsigned ring, coef_t, coef_w, phase, whist, bhist, ghist, lmask, gmask, gpre, xch, misc,
         srcidx, bars, total;
-    int stage_rows;    // compaction rows per CTA per round
-    unsigned regionA;  // bytes of sc + ring (reused as the compaction stage)
+    int stage_rows;    // compaction rows per CTA per round (staged in the ring)
 };
 
 __host__ __device__ inline unsigned align_up(unsigned x, unsigned a) { return (x + a - 1) / a * a; }
@@ -110,13 +116,10 @@ __host__ __device__ inline Layout make_layout(int D, int G, int nslot, int kpc, 
     unsigned o = 0;
     const int F = D / 2;
     const int nwl = kpc / 32;
-    L.sc = o;
-    o = align_up(o + (unsigned)kpc * G * 4u, 128);
     L.ring = o;
     o = align_up(o + (unsigned)kWarps * nslot * kStageRows * D * 2u, 128);
-    L.regionA = o;
     const unsigned row_bytes = (unsigned)D * 2u * 2u + 4u;
-    int S = (int)(L.regionA / row_bytes);
+    int S = (int)(o / row_bytes);
     S = S / 16 * 16;
     L.stage_rows = S;
     L.coef_t = o;
@@ -139,8 +142,8 @@ __host__ __device__ inline Layout make_layout(int D, int G, int nslot, int kpc, 
     o = align_up(o + ((unsigned)cs * nwl + 1u) * 4u, 16);
     L.xch = o;
     o = align_up(o + sizeof(Xch), 16);
-    L.misc = o;  // block-reduction scratch: kWarps * 8 doubles + broadcast words
-    o = align_up(o + (unsigned)kWarps * 8u * 8u + 64u * 4u + 8u * 16u, 16);
+    L.misc = o;  // block-reduction scratch: kWarps + 1 doubles, 64 ints, 32 floats
+    o = align_up(o + (unsigned)(kWarps + 1) * 8u + 64u * 4u + 32u * 4u, 16);
     L.srcidx = o;
     o = align_up(o + (unsigned)(S > 0 ? S : 1) * 4u, 16);
     L.bars = o;
@@ -169,24 +172,24 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, unsigned bytes) {
                  : "memory");
 }
 
+// One potentially blocking test of the barrier phase: the hardware suspends the warp until
+// the phase completes or the time hint runs out, so waiting costs no issue slots.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
     unsigned ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(kWaitSuspendNs)
         : "memory");
     return ok != 0;
 }
 
-// Bounded wait: returns false if the phase did not complete within the poll limit.
+// Bounded wait (about one second at most): returns false if the phase never completed.
 __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
-    for (long long i = 0; i < kWaitLimit; ++i) {
+    for (int i = 0; i < kWaitTries; ++i)
         if (mbar_try_wait(bar, parity)) return true;
-        if (i > 64) __nanosleep(256);
-    }
     return false;
 }
 
@@ -194,14 +197,35 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// 1-D bulk copy global -> shared, completion signalled on an mbarrier (no multicast).
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+__device__ __forceinline__ uint64_t policy_evict_last() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+// 1-D bulk copy global -> shared, completion signalled on an mbarrier, with an L2
+// eviction-priority hint (no multicast).
 __device__ __forceinline__ void tma_load_1d(void *dst_smem, const void *src_gmem, unsigned bytes,
-                                            uint64_t *bar) {
+                                            uint64_t *bar, uint64_t policy) {
     asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_u32(dst_smem)),
-        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar))
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(smem_u32(dst_smem)),
+        "l"(src_gmem), "r"(bytes), "r"(smem_u32(bar)), "l"(policy)
         : "memory");
+}
+
+__device__ __forceinline__ void st_hint(float *p, float v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
+}
+
+__device__ __forceinline__ void st_hint_u32(unsigned *p, unsigned v, uint64_t policy) {
+    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
 }
 
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
@@ -214,16 +238,6 @@ __device__ __forceinline__ void cp_async4(void *dst_smem, const void *src) {
 
 __device__ __forceinline__ void cp_async_wait_all() {
     asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
-}
-
-// acc += a * b on two fp32 lanes at once (sm_100 packed FMA).
-__device__ __forceinline__ void ffma2(float2 &acc, float2 a, float2 b) {
-    unsigned long long A, B, C;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(A) : "f"(a.x), "f"(a.y));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(B) : "f"(b.x), "f"(b.y));
-    asm("mov.b64 %0, {%1, %2};" : "=l"(C) : "f"(acc.x), "f"(acc.y));
-    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(C) : "l"(A), "l"(B));
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(acc.x), "=f"(acc.y) : "l"(C));
 }
 
 __device__ __forceinline__ float sqrt_approx(float x) {
@@ -271,47 +285,50 @@ __device__ __forceinline__ int select_bit(unsigned m, int k) {
     return pos;
 }
 
-// Exclusive scan of n (<= 4 * kThreads) ints in place in shared memory; returns the total.
+// Exclusive scan of n ints in place in shared memory (any n); returns the total.
 // All threads of the block must call it.
-__device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 1 ints */) {
+__device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 ints */) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int PER = 4;
-    int v[PER];
-    int local = 0;
+    int carry = 0;
+    for (int base = 0; base < n; base += PER * kThreads) {
+        int v[PER];
+        int local = 0;
 #pragma unroll
-    for (int k = 0; k < PER; ++k) {
-        const int i = tid * PER + k;
-        v[k] = i < n ? a[i] : 0;
-        local += v[k];
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-    }
-    if (lane == 31) scratch[warp] = incl;
-    __syncthreads();
-    if (tid == 0) {
-        int run = 0;
-        for (int w = 0; w < kWarps; ++w) {
-            const int x = scratch[w];
-            scratch[w] = run;
-            run += x;
+        for (int k = 0; k < PER; ++k) {
+            const int i = base + tid * PER + k;
+            v[k] = i < n ? a[i] : 0;
+            local += v[k];
         }
-        scratch[kWarps] = run;
-    }
-    __syncthreads();
-    int ex = scratch[warp] + incl - local;
+        int incl = local;
 #pragma unroll
-    for (int k = 0; k < PER; ++k) {
-        const int i = tid * PER + k;
-        if (i < n) a[i] = ex;
-        ex += v[k];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        if (lane == 31) scratch[warp] = incl;
+        __syncthreads();
+        if (tid == 0) {
+            int run = 0;
+            for (int w = 0; w < kWarps; ++w) {
+                const int x = scratch[w];
+                scratch[w] = run;
+                run += x;
+            }
+            scratch[kWarps] = run;
+        }
+        __syncthreads();
+        int ex = carry + scratch[warp] + incl - local;
+#pragma unroll
+        for (int k = 0; k < PER; ++k) {
+            const int i = base + tid * PER + k;
+            if (i < n) a[i] = ex;
+            ex += v[k];
+        }
+        carry += scratch[kWarps];
+        __syncthreads();
     }
-    const int total = scratch[kWarps];
-    __syncthreads();
-    return total;
+    return carry;
 }
 
 // Sum of one double per thread over the block; result valid in every thread.
@@ -384,6 +401,23 @@ __device__ __forceinline__ void unpack_pairs(const unsigned (&w)[NP], float2 (&x
     }
 }
 
+// The G scores of one key (16-byte aligned rows of G floats).
+template <int G>
+__device__ __forceinline__ void load_scores(const float *p, float (&v)[G]) {
+    if constexpr (G >= 4) {
+#pragma unroll
+        for (int q = 0; q < G / 4; ++q) {
+            const float4 x = *reinterpret_cast<const float4 *>(p + 4 * q);
+            v[4 * q] = x.x; v[4 * q + 1] = x.y; v[4 * q + 2] = x.z; v[4 * q + 3] = x.w;
+        }
+    } else if constexpr (G == 2) {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        v[0] = x.x; v[1] = x.y;
+    } else {
+        v[0] = *p;
+    }
+}
+
 // Dim index (within the lane's DH-dim chunk) of element e (0 = .x, 1 = .y) of pair p.
 template <int LAYOUT>
 __host__ __device__ constexpr int pair_dim(int p, int e) {
@@ -391,26 +425,29 @@ __host__ __device__ constexpr int pair_dim(int p, int e) {
 }
 
 // ---------------------------------------------------------------------------------
-// The fused kernel. Grid: (cs * n_units) CTAs in clusters of cs; block: kThreads.
+// The fused kernel. Grid: n_clusters * cs CTAs (clusters of cs), persistent over units.
 // ---------------------------------------------------------------------------------
 template <int D, int G, int LAYOUT>
-__global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
+__global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const Args a) {
     constexpr int F = D / 2;
     using GE = Geo<D, G>;
     constexpr int DH = GE::DH;
     constexpr int LPK = GE::LPK;
     constexpr int KPP = GE::KPP;
+    constexpr int NP = GE::NP;
     constexpr unsigned FULL = 0xffffffffu;
+    constexpr unsigned kStageBytes = kStageRows * D * 2;
 
     extern __shared__ __align__(128) unsigned char smem[];
     cg::cluster_group cluster = cg::this_cluster();
     const int cs = a.cs;
     const int crank = (int)cluster.block_rank();
-    const int unit = blockIdx.x / cs;
+    const int cid = blockIdx.x / cs;
+    const int n_clusters = gridDim.x / cs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const Layout Ly = make_layout(D, G, a.nslot, a.kpc_max, cs);
+    const int nslot = a.nslot;
+    const Layout Ly = make_layout(D, G, nslot, a.kpc_max, cs);
 
-    float *sc = reinterpret_cast<float *>(smem + Ly.sc);
     unsigned char *ring = smem + Ly.ring;
     float *coef_t = reinterpret_cast<float *>(smem + Ly.coef_t);
     float *coef_w = reinterpret_cast<float *>(smem + Ly.coef_w);
@@ -423,54 +460,89 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
     int *gpre = reinterpret_cast<int *>(smem + Ly.gpre);
     Xch *xch = reinterpret_cast<Xch *>(smem + Ly.xch);
     double *dscratch = reinterpret_cast<double *>(smem + Ly.misc);
-    int *iscratch = reinterpret_cast<int *>(smem + Ly.misc + kWarps * 8 * 8);
-    float *bcast = reinterpret_cast<float *>(smem + Ly.misc + kWarps * 8 * 8 + 64 * 4);
+    int *iscratch = reinterpret_cast<int *>(smem + Ly.misc + (kWarps + 1) * 8);
+    float *bcast = reinterpret_cast<float *>(smem + Ly.misc + (kWarps + 1) * 8 + 64 * 4);
     int *srcidx = reinterpret_cast<int *>(smem + Ly.srcidx);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Ly.bars);
 
-    const int g = unit % a.n_kv;
-    const int s = (unit / a.n_kv) % a.batch;
-    const int lr = unit / (a.n_kv * a.batch);
-    const int layer = a.layer_begin + lr;
-    const int Hq = a.n_kv * G;
-    const int N = __ldg(a.lens + s);
-    bool talked = false;  // did this cluster use distributed shared memory
+    __shared__ double part_d[kMaxCluster][8], part_q[kMaxCluster][8];
+    __shared__ double w_s[kWarps][8], w_q[kWarps][8];
+    __shared__ float w_lo[kWarps][8], w_hi[kWarps][8];
+    __shared__ float part_lo[kMaxCluster][8], part_hi[kMaxCluster][8];
+    __shared__ int part_fail[kMaxCluster];
+    __shared__ float muf_s[8], inv_s[8];
+    __shared__ int anyfail_s, sel_s[3];
 
-    // ---- validation: every CTA of the cluster reaches the same verdict --------------
-    int bad = (N < 0 || N > a.cap_u) ? kDevLenGtCap : 0;
-    if (!bad && a.paged) {
-        const int np = (N + a.page_size - 1) / a.page_size;
-        int mine = 0;
-        for (int p = tid; p < np; p += kThreads) {
-            const int pg = __ldg(a.block_table + (long long)s * a.max_pages + p);
-            if (pg < 0 || pg >= a.n_pages) mine = 1;
-        }
-        if (__syncthreads_or(mine)) bad = kDevBadPage;
+    // this cluster's scratch slot: scores [cap_u][G], then order keys [cap_u]
+    float *sc = a.scratch + (long long)cid * a.slot_floats;
+    unsigned *ukey = reinterpret_cast<unsigned *>(sc + (long long)a.cap_u * G);
+    const uint64_t pol_first = policy_evict_first();
+    const uint64_t pol_last = policy_evict_last();
+
+    // per-warp TMA buffers; the counters run on across units so that slot and phase
+    // parity stay in step with the barriers
+    if (lane == 0) {
+        for (int k = 0; k < nslot; ++k) mbar_init(bars + warp * nslot + k, 1);
+        mbar_init_fence();
     }
-    if (bad) {
-        if (crank == 0 && tid == 0) {
+    __syncwarp();
+    // ring bookkeeping, advanced incrementally (no division by the runtime slot count):
+    // the producer fills slot wr_slot; the consumer waits on slot rd_slot for phase rd_phase
+    int wr_slot = 0, rd_slot = 0;
+    unsigned rd_phase = 0;
+
+    // lane geometry (fixed for the whole launch)
+    const int sub = lane % LPK;
+    const int kw = lane / LPK;
+    int hx = 0;
+    {
+        int cnt = G;
+#pragma unroll
+        for (int m = LPK / 2; m >= 1; m >>= 1) {
+            if (cnt > 1) {
+                const int half = cnt / 2;
+                if (lane & m) hx |= half;
+                cnt = half;
+            }
+        }
+    }
+    const bool writer = (sub & (LPK / G - 1)) == 0;
+    const int Hq = a.n_kv * G;
+
+    for (int unit = cid; unit < a.n_units; unit += n_clusters) {
+        const int g = unit % a.n_kv;
+        const int s = (unit / a.n_kv) % a.batch;
+        const int lr = unit / (a.n_kv * a.batch);
+        const int layer = a.layer_begin + lr;
+        const int N = __ldg(a.lens + s);
+
+        // ---- validation: every CTA of the cluster reaches the same verdict ----------
+        int bad = (N < 0 || N > a.cap_u) ? kDevLenGtCap : 0;
+        if (!bad && a.paged) {
+            const int np = (N + a.page_size - 1) / a.page_size;
+            int mine = 0;
+            for (int p = tid; p < np; p += kThreads) {
+                const int pg = __ldg(a.block_table + (long long)s * a.max_pages + p);
+                if (pg < 0 || pg >= a.n_pages) mine = 1;
+            }
+            if (__syncthreads_or(mine)) bad = kDevBadPage;
+        }
+        if (bad && crank == 0 && tid == 0) {
             record_status(a.status, bad, unit);
             if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
-    }
-    const bool work = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
+        const bool work = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
+        if (!work) continue;  // uniform over the cluster: no cluster barrier is skipped unevenly
 
-    if (work) {
-        talked = true;
         const int kpc = ((N + cs - 1) / cs + 31) / 32 * 32;
         const int begin = crank * kpc;
         const int n_local = max(0, min(N - begin, kpc));
         const int nst = (n_local + kStageRows - 1) / kStageRows;
-        const int nslot = a.nslot;
-        constexpr unsigned kStageBytes = kStageRows * D * 2;
+        const int my_stages = warp < nst ? (nst - warp + kWarps - 1) / kWarps : 0;
 
         // ---- start streaming this CTA's keys (TMA bulk copies, per-warp buffers) -----
-        if (lane == 0) {
-            for (int k = 0; k < nslot; ++k) mbar_init(bars + warp * nslot + k, 1);
-            mbar_init_fence();
-        }
-        __syncwarp();
-        auto issue = [&](int st, int slot) {
+        auto issue = [&](int st) {
+            const int slot = wr_slot;
             const int row0 = st * kStageRows;
             const int nrows = min(kStageRows, n_local - row0);
             const long long r = row_of(a, lr, s, g, begin + row0);
@@ -478,12 +550,14 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             fence_proxy_async_smem();
             mbar_expect_tx(bar, (unsigned)nrows * D * 2u);
             tma_load_1d(ring + (size_t)(warp * nslot + slot) * kStageBytes, a.K + r * D,
-                        (unsigned)nrows * D * 2u, bar);
+                        (unsigned)nrows * D * 2u, bar, pol_first);
         };
-        if (lane == 0) {
-            for (int k = 0; k < nslot; ++k) {
-                const int st = warp + k * kWarps;
-                if (st < nst) issue(st, k);
+        __syncthreads();  // the ring is free (previous unit's staging reads are done)
+        {
+            const int pre = min(nslot, my_stages);
+            for (int k = 0; k < pre; ++k) {
+                if (lane == 0) issue(warp + k * kWarps);
+                if (++wr_slot == nslot) wr_slot = 0;
             }
         }
 
@@ -510,22 +584,6 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
         }
         __syncthreads();
 
-        // ---- lane geometry and register-resident coefficients ----------------------
-        const int sub = lane % LPK;
-        const int kw = lane / LPK;
-        int hx = 0;
-        {
-            int cnt = G;
-#pragma unroll
-            for (int m = LPK / 2; m >= 1; m >>= 1) {
-                if (cnt > 1) {
-                    const int half = cnt / 2;
-                    if (lane & m) hx |= half;
-                    cnt = half;
-                }
-            }
-        }
-        constexpr int NP = GE::NP;
         // register-resident coefficients, in the pair order the unpack produces
         float2 ca[G][NP], cb[G][NP], cw[G][NP];
 #pragma unroll
@@ -536,55 +594,56 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                 const int d0 = pair_dim<LAYOUT>(p, 0), d1 = pair_dim<LAYOUT>(p, 1);
                 ca[i][p] = make_float2(coef_t[hq * D + sub * DH + d0], coef_t[hq * D + sub * DH + d1]);
                 cb[i][p] = make_float2(coef_t[hq * D + F + sub * DH + d0], coef_t[hq * D + F + sub * DH + d1]);
-                // norm pairs: half layout -> bands (sub*DH + 2p, +1); interleaved -> pairs
-                // 0..NP/2-1 come from the first-half chunk, the rest from the second
-                int b0, b1;
+                int b0;
                 if (LAYOUT == 0) {
                     b0 = sub * DH + 2 * p;
-                    b1 = b0 + 1;
                 } else {
                     const int base = (p < NP / 2) ? sub * (DH / 2) : D / 4 + sub * (DH / 2);
                     const int q = (p < NP / 2) ? p : p - NP / 2;
                     b0 = base + 2 * q;
-                    b1 = b0 + 1;
                 }
-                cw[i][p] = make_float2(coef_w[hq * F + b0], coef_w[hq * F + b1]);
+                cw[i][p] = make_float2(coef_w[hq * F + b0], coef_w[hq * F + b0 + 1]);
             }
         }
-        const bool writer = (sub & (LPK / G - 1)) == 0;
         float *raw_row = nullptr;
         if (a.raw)
             raw_row = a.raw + (((long long)lr * a.batch + s) * Hq + (long long)g * G + hx) * (long long)a.cap_u + begin;
+        float *sc_local = sc + (long long)begin * G;
 
         // ---- score loop ----------------------------------------------------------------
+        // writer lanes also gather their head's moments (fp64 sum and sum of squares, fp32
+        // min and max) so that the scores are read back only once, for the z-score
+        double m_s = 0.0, m_q = 0.0;
+        float m_lo = __int_as_float(0x7f800000), m_hi = -__int_as_float(0x7f800000);
         int fail = 0;
-        for (int k = 0;; ++k) {
+        for (int k = 0; k < my_stages; ++k) {
             const int st = warp + k * kWarps;
-            if (st >= nst) break;
-            const int slot = k % nslot;
-            const bool landed = __all_sync(FULL, mbar_wait_bounded(bars + warp * nslot + slot,
-                                                                    (unsigned)((k / nslot) & 1)));
+            const int slot = rd_slot;
+            const bool landed = __all_sync(FULL, mbar_wait_bounded(bars + warp * nslot + slot, rd_phase));
             if (!landed) {
                 // give the copies this warp still has in flight a bounded chance to land
-                // before the buffers are abandoned
-                for (int j = 1; j < nslot; ++j) {
-                    const int kk = k + j;
-                    if (warp + kk * kWarps < nst)
-                        (void)mbar_wait_bounded(bars + warp * nslot + kk % nslot, (unsigned)((kk / nslot) & 1));
+                int sl = slot;
+                unsigned ph = rd_phase;
+                for (int j = k + 1; j < min(my_stages, k + nslot); ++j) {
+                    if (++sl == nslot) { sl = 0; ph ^= 1u; }
+                    (void)mbar_wait_bounded(bars + warp * nslot + sl, ph);
                 }
                 fail = 1;
                 break;
             }
             const uint16_t *stage =
                 reinterpret_cast<const uint16_t *>(ring + (size_t)(warp * nslot + slot) * kStageBytes);
-#pragma unroll 2
+            const uint16_t *lane_a = stage + kw * D + sub * DH;
+            const int li0 = st * kStageRows + kw;
+            float *sc_pass = sc_local + li0 * G + hx;
+            float *raw_pass = raw_row ? raw_row + li0 : nullptr;
+            const int valid = n_local - li0;  // key of pass p is valid when p * KPP < valid
+#pragma unroll
             for (int pass = 0; pass < kStageRows / KPP; ++pass) {
-                const int r = pass * KPP + kw;
-                const int li = st * kStageRows + r;
-                const uint16_t *row = stage + r * D;
+                const uint16_t *row = lane_a + pass * KPP * D;
                 unsigned wa[DH / 2], wb[DH / 2];
-                load_chunk<DH>(row + sub * DH, wa);
-                load_chunk<DH>(row + F + sub * DH, wb);
+                load_chunk<DH>(row, wa);
+                load_chunk<DH>(row + F, wb);
                 float2 xa[NP], xb[NP], nb[NP];
                 unpack_pairs<NP, LAYOUT>(wa, xa);
                 unpack_pairs<NP, LAYOUT>(wb, xb);
@@ -633,14 +692,22 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                         }
                     }
                 }
-                if (writer && li < n_local) {
-                    sc[li * G + hx] = v[0];
-                    if (raw_row) raw_row[li] = v[0];
+                if (writer && pass * KPP < valid) {
+                    st_hint(sc_pass + pass * KPP * G, v[0], pol_last);
+                    if (raw_pass) raw_pass[pass * KPP] = v[0];
+                    const double dv = (double)v[0];
+                    m_s += dv;
+                    m_q = fma(dv, dv, m_q);
+                    m_lo = fminf(m_lo, v[0]);
+                    m_hi = fmaxf(m_hi, v[0]);
                 }
             }
             __syncwarp();
-            const int nxt = st + nslot * kWarps;
-            if (lane == 0 && nxt < nst) issue(nxt, slot);
+            if (++rd_slot == nslot) { rd_slot = 0; rd_phase ^= 1u; }
+            if (k + nslot < my_stages) {
+                if (lane == 0) issue(warp + (k + nslot) * kWarps);
+                if (++wr_slot == nslot) wr_slot = 0;
+            }
         }
         if (__syncthreads_or(fail)) {
             if (tid == 0) {
@@ -650,54 +717,49 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             fail = 1;
         }
 
-        // ---- per-head moments over the whole unit (two passes, fp64, cluster-wide) -----
+        // ---- per-head moments over the whole unit (fp64, cluster-wide) ---------------------
+        // Lanes that hold the same head differ only in their key-group bits: fold those in
+        // a fixed order, then the warps in order, then the cluster's CTAs in rank order, so
+        // that every CTA obtains bit-identical mu and sigma.
         {
-            double sum[G];
-            float mn[G], mx[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) { sum[h] = 0.0; mn[h] = __int_as_float(0x7f800000); mx[h] = -mn[h]; }
-            for (int i = tid; i < n_local; i += kThreads) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float x = sc[i * G + h];
-                    sum[h] += (double)x;
-                    mn[h] = fminf(mn[h], x);
-                    mx[h] = fmaxf(mx[h], x);
-                }
+            for (int o = LPK; o < 32; o <<= 1) {
+                m_s += __shfl_xor_sync(FULL, m_s, o);
+                m_q += __shfl_xor_sync(FULL, m_q, o);
+                m_lo = fminf(m_lo, __shfl_xor_sync(FULL, m_lo, o));
+                m_hi = fmaxf(m_hi, __shfl_xor_sync(FULL, m_hi, o));
             }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const double t = block_sum_f64(sum[h], dscratch);
-                float lo = mn[h], hi = mx[h];
-#pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) {
-                    lo = fminf(lo, __shfl_xor_sync(FULL, lo, o));
-                    hi = fmaxf(hi, __shfl_xor_sync(FULL, hi, o));
+            if (kw == 0 && writer) {
+                w_s[warp][hx] = m_s;
+                w_q[warp][hx] = m_q;
+                w_lo[warp][hx] = m_lo;
+                w_hi[warp][hx] = m_hi;
+            }
+            __syncthreads();
+            if (tid < G) {
+                double ts_ = 0.0, tq_ = 0.0;
+                float lo = __int_as_float(0x7f800000), hi = -lo;
+                for (int w = 0; w < kWarps; ++w) {
+                    ts_ += w_s[w][tid];
+                    tq_ += w_q[w][tid];
+                    lo = fminf(lo, w_lo[w][tid]);
+                    hi = fmaxf(hi, w_hi[w][tid]);
                 }
-                if (lane == 0) { bcast[2 * warp] = lo; bcast[2 * warp + 1] = hi; }
-                __syncthreads();
-                if (tid == 0) {
-                    float l2 = bcast[0], h2 = bcast[1];
-                    for (int w = 1; w < kWarps; ++w) { l2 = fminf(l2, bcast[2 * w]); h2 = fmaxf(h2, bcast[2 * w + 1]); }
-                    xch->sum[h] = t; xch->mn[h] = l2; xch->mx[h] = h2;
-                }
-                __syncthreads();
+                xch->sum[tid] = ts_;
+                xch->m2[tid] = tq_;
+                xch->mn[tid] = lo;
+                xch->mx[tid] = hi;
             }
             if (tid == 0) xch->fail = fail;
         }
         cluster.sync();
         // every CTA gathers the cluster's partials (one remote load per thread, all in
-        // flight together) and folds them in rank order: identical mu in every CTA
-        __shared__ double part_d[kMaxCluster][8];
-        __shared__ float part_lo[kMaxCluster][8], part_hi[kMaxCluster][8];
-        __shared__ int part_fail[kMaxCluster];
-        __shared__ double mu_s[8];
-        __shared__ float muf_s[8], inv_s[8];
-        __shared__ int flat_s[8], anyfail_s;
+        // flight together) and folds them in rank order
         for (int idx = tid; idx < cs * G; idx += kThreads) {
             const int c = idx / G, h = idx % G;
             const Xch *r = cluster.map_shared_rank(xch, c);
             part_d[c][h] = r->sum[h];
+            part_q[c][h] = r->m2[h];
             part_lo[c][h] = r->mn[h];
             part_hi[c][h] = r->mx[h];
             if (h == 0) part_fail[c] = r->fail;
@@ -705,15 +767,22 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
         __syncthreads();
         if (tid < G) {
             const int h = tid;
-            double tot = 0.0;
+            double tot = 0.0, totq = 0.0;
             float lo = __int_as_float(0x7f800000), hi = -lo;
             for (int c = 0; c < cs; ++c) {
                 tot += part_d[c][h];
+                totq += part_q[c][h];
                 lo = fminf(lo, part_lo[c][h]);
                 hi = fmaxf(hi, part_hi[c][h]);
             }
-            mu_s[h] = tot / (double)N;
-            flat_s[h] = !(hi > lo);
+            // population variance from fp64 sums (fp32 scores: no cancellation to fear at
+            // fp64 precision); a head whose scores are all equal is flat
+            const double mu = tot / (double)N;
+            const double var = fmax(totq / (double)N - mu * mu, 0.0);
+            const double sigma = sqrt(var);
+            const bool flat = !(hi > lo);
+            muf_s[h] = (float)mu;
+            inv_s[h] = (flat || !(sigma > 0.0)) ? 0.f : (float)(1.0 / sigma);
         }
         if (tid == 32) {
             int f = 0;
@@ -721,71 +790,65 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             anyfail_s = f;
         }
         __syncthreads();
-        {
-            double m2[G];
-#pragma unroll
-            for (int h = 0; h < G; ++h) m2[h] = 0.0;
-            for (int i = tid; i < n_local; i += kThreads) {
-#pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const double dlt = (double)sc[i * G + h] - mu_s[h];
-                    m2[h] += dlt * dlt;
-                }
-            }
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const double t = block_sum_f64(m2[h], dscratch);
-                if (tid == 0) xch->m2[h] = t;
-            }
-        }
-        cluster.sync();
-        for (int idx = tid; idx < cs * G; idx += kThreads) {
-            const int c = idx / G, h = idx % G;
-            part_d[c][h] = cluster.map_shared_rank(xch, c)->m2[h];
-        }
-        __syncthreads();
-        if (tid < G) {
-            const int h = tid;
-            double tot = 0.0;
-            for (int c = 0; c < cs; ++c) tot += part_d[c][h];
-            const double sigma = sqrt(tot / (double)N);
-            muf_s[h] = (float)mu_s[h];
-            inv_s[h] = (flat_s[h] || !(sigma > 0.0)) ? 0.f : (float)(1.0 / sigma);
-        }
-        __syncthreads();
 
-        // ---- z-score, max over the group; the order key replaces the key's first score --
+        // ---- z-score, max over the group, order key --------------------------------------
+        // The order keys live in the (now idle) TMA ring when they fit, else in the scratch
+        // slot; the first radix digit's histogram is built on the way.
         float *zrow = a.zmax ? a.zmax + (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + begin
                              : nullptr;
-        for (int i = tid; i < n_local; i += kThreads) {
-            float z = -__int_as_float(0x7f800000);
-#pragma unroll
-            for (int h = 0; h < G; ++h) {
-                const float zh = (sc[i * G + h] - muf_s[h]) * inv_s[h];
-                z = fmaxf(z, zh);
+        const bool keys_on_chip = (long long)n_local * 4 <= (long long)kWarps * nslot * kStageBytes;
+        unsigned *uk = keys_on_chip ? reinterpret_cast<unsigned *>(ring) : ukey + begin;
+        const bool selecting = a.mode == kModePrune && !anyfail_s;
+        {
+            unsigned *wh = whist + warp * kBins;
+            if (selecting) {
+                for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
+                __syncwarp();
             }
-            z = z + 0.0f;  // -0 -> +0
-            if (zrow) zrow[i] = z;
-            reinterpret_cast<unsigned *>(sc)[i * G] = float_key(z);
+            const int lim = (n_local + 31) / 32 * 32;
+#pragma unroll 4
+            for (int i = tid; i < lim; i += kThreads) {
+                const bool in = i < n_local;
+                unsigned key = 0u;
+                if (in) {
+                    float sv[G];
+                    load_scores<G>(sc_local + i * G, sv);
+                    float z = -__int_as_float(0x7f800000);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) z = fmaxf(z, (sv[h] - muf_s[h]) * inv_s[h]);
+                    z = z + 0.0f;  // -0 -> +0
+                    if (zrow) zrow[i] = z;
+                    key = float_key(z);
+                    uk[i] = key;
+                }
+                if (selecting) {
+                    const unsigned bin = key >> 24;
+                    const unsigned act = __ballot_sync(FULL, in);
+                    if (in) {
+                        const unsigned peers = __match_any_sync(act, bin);
+                        if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
+                    }
+                }
+            }
         }
         __syncthreads();
-        const unsigned *ukey = reinterpret_cast<const unsigned *>(sc);
 
-        if (a.mode == kModePrune && !anyfail_s) {
+        if (selecting) {
             // ---- radix select of the B-th largest key, cluster-wide ------------------------
             unsigned prefix = 0u, pmask = 0u;
             int need = a.budget;
             bool resolved = false;
-            __shared__ int sel_s[3];
             for (int pass = 0; pass < 4 && !resolved; ++pass) {
                 const int shift = 24 - 8 * pass;
                 unsigned *wh = whist + warp * kBins;
-                for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
-                __syncwarp();
-                const int lim = (n_local + 31) / 32 * 32;
+                const int lim = pass == 0 ? 0 : (n_local + 31) / 32 * 32;  // pass 0 built above
+                if (pass > 0) {
+                    for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
+                    __syncwarp();
+                }
                 for (int i = tid; i < lim; i += kThreads) {
                     const bool in = i < n_local;
-                    const unsigned u = in ? ukey[i * G] : 0u;
+                    const unsigned u = in ? uk[i] : 0u;
                     const bool m = in && ((u & pmask) == prefix);
                     const unsigned bin = (u >> shift) & 255u;
                     const unsigned act = __ballot_sync(FULL, m);
@@ -812,14 +875,13 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                     unsigned c = 0u;
 #pragma unroll
                     for (int r = 0; r < kMaxCluster; ++r) c += part[r];
-                    gh[kBins - 1 - b] = (int)c;  // reversed: index 0 is the top bin
+                    gh[kBins - 1 - b] = (int)c;
                 }
                 __syncthreads();
-                // inclusive scan over reversed bins
                 if (warp == 0) {
                     int run = 0;
                     for (int base = 0; base < kBins; base += 32) {
-                        int x = gh[base + lane];
+                        const int x = gh[base + lane];
                         int incl = x;
 #pragma unroll
                         for (int o = 1; o < 32; o <<= 1) {
@@ -854,7 +916,7 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             if (tie) {
                 for (int wi = warp; wi < nwl; wi += kWarps) {
                     const int i = wi * 32 + lane;
-                    const bool eq = i < n_local && ukey[i * G] == prefix;
+                    const bool eq = i < n_local && uk[i] == prefix;
                     const unsigned bb = __ballot_sync(FULL, eq);
                     if (lane == 0) tw[wi] = __popc(bb);
                 }
@@ -873,7 +935,7 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
             for (int wi = warp; wi < nwl; wi += kWarps) {
                 const int i = wi * 32 + lane;
                 const bool in = i < n_local;
-                const unsigned u = in ? ukey[i * G] : 0u;
+                const unsigned u = in ? uk[i] : 0u;
                 const bool gt = in && (u & pmask) > prefix;
                 const bool eq = in && (u & pmask) == prefix;
                 bool keep = gt || (eq && !tie);
@@ -895,24 +957,13 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
                 gpre[wg] = __popc(m);
             }
             __syncthreads();
-            // nwt can exceed 4 * kThreads for tiny kpc * large cs only when nwt > 1024;
-            // the host keeps cs * kpc <= 32768 * 4 so nwt <= 4096 -> scan in 4 chunks
-            {
-                int run = 0;
-                for (int base = 0; base < nwt; base += 4 * kThreads) {
-                    const int n = min(4 * kThreads, nwt - base);
-                    const int tot = block_exclusive_scan(gpre + base, n, iscratch);
-                    for (int q = tid; q < n; q += kThreads) gpre[base + q] += run;
-                    __syncthreads();
-                    run += tot;
-                }
-                if (tid == 0) gpre[nwt] = run;
-                __syncthreads();
-            }
+            const int total = block_exclusive_scan(gpre, nwt, iscratch);
+            if (tid == 0) gpre[nwt] = total;
+            __syncthreads();
             const int M = a.budget;
             // the mask must hold exactly M keys; anything else is an internal error and the
             // unit is left untouched rather than copied from a wrong index
-            const bool count_ok = gpre[nwt] == M;
+            const bool count_ok = total == M;
             if (!count_ok && crank == 0 && tid == 0) {
                 record_status(a.status, kDevInternal, unit);
                 if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
@@ -920,7 +971,7 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
 
             // ---- in-place stable compaction in ascending destination rounds ---------------
             const int S = Ly.stage_rows;
-            uint16_t *stK = reinterpret_cast<uint16_t *>(smem);  // region A
+            uint16_t *stK = reinterpret_cast<uint16_t *>(ring);
             uint16_t *stV = stK + (size_t)S * D;
             int32_t *stP = reinterpret_cast<int32_t *>(stV + (size_t)S * D);
             constexpr int LPR = D / 8;  // lanes per row (16 bytes each)
@@ -966,10 +1017,10 @@ __global__ void __launch_bounds__(kThreads, 1) tri_fused_kernel(const Args a) {
         } else if (a.mode == kModePrune && anyfail_s) {
             if (crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
+        // the next unit reuses this CTA's exchange buffers and masks: nobody may still be
+        // reading them
+        cluster.sync();
     }
-
-    // nobody leaves while a peer may still read its shared memory
-    if (talked) cluster.sync();
 
     // ---- the last CTA to finish publishes the new lengths ------------------------------
     if (a.mode == kModePrune && a.lens_out) {
