@@ -161,6 +161,14 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+def workload_spec(args):
+    import tri_synth as ts
+    spec = ts.WORKLOADS[args.workload]
+    if args.layers:
+        spec = ts.replace(spec, n_layers=args.layers)
+    return spec
+
+
 # ---------------------------------------------------------------------------------------
 # our arm
 # ---------------------------------------------------------------------------------------
@@ -174,7 +182,7 @@ def run_ours(args, rank, world, dist_mod):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
-    spec = ts.WORKLOADS[args.workload]
+    spec = workload_spec(args)
     B = spec.budget
     cache = ts.make_cache(spec, seed=1000 + rank, device=dev)
     torch.cuda.synchronize()
@@ -402,7 +410,7 @@ def run_reference(args, rank, world):
     import torch
 
     import tri_synth as ts
-    spec = ts.WORKLOADS[args.workload]
+    spec = workload_spec(args)
     # only the host copy of a bounded sample is needed: draw the cache on the GPU when one
     # is present (the full workload is ~19 GB), else draw it on the CPU
     dev = "cuda" if torch.cuda.is_available() else "cpu"
@@ -438,6 +446,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--layers", type=int, default=0,
+                    help="override the workload's layer count (smaller cases for profiling)")
     ap.add_argument("--cluster-size", type=int, default=0)
     ap.add_argument("--buffers", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)

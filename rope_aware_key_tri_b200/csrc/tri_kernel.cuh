@@ -331,24 +331,6 @@ __device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 in
     return carry;
 }
 
-// Sum of one double per thread over the block; result valid in every thread.
-__device__ double block_sum_f64(double x, double *scratch /* kWarps + 1 */) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
-    if (lane == 0) scratch[warp] = x;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        double r = 0.0;
-        for (int w = 0; w < kWarps; ++w) r += scratch[w];
-        scratch[kWarps] = r;
-    }
-    __syncthreads();
-    const double r = scratch[kWarps];
-    __syncthreads();
-    return r;
-}
-
 // ---------------------------------------------------------------------------------
 // Per-key slice geometry. A key of D dims is split over LPK lanes; each lane holds DH
 // consecutive dims from the first half of the row and the DH dims D/2 further on, i.e.
@@ -459,9 +441,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
     unsigned *gmask = reinterpret_cast<unsigned *>(smem + Ly.gmask);
     int *gpre = reinterpret_cast<int *>(smem + Ly.gpre);
     Xch *xch = reinterpret_cast<Xch *>(smem + Ly.xch);
-    double *dscratch = reinterpret_cast<double *>(smem + Ly.misc);
     int *iscratch = reinterpret_cast<int *>(smem + Ly.misc + (kWarps + 1) * 8);
-    float *bcast = reinterpret_cast<float *>(smem + Ly.misc + (kWarps + 1) * 8 + 64 * 4);
     int *srcidx = reinterpret_cast<int *>(smem + Ly.srcidx);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + Ly.bars);
 
@@ -969,51 +949,62 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
             }
 
-            // ---- in-place stable compaction in ascending destination rounds ---------------
+            // ---- in-place stable compaction ------------------------------------------------
+            // Kept rows never move to a higher slot. The only sources a write to [0, M) can
+            // clobber are the kept rows below slot M (the first q kept rows, which land in
+            // [0, q)). Those move in ascending destination rounds: every CTA first copies its
+            // round's sources into shared memory, the cluster synchronises, then all write.
+            // The other M - q kept rows come from slots >= M, which no write touches; once the
+            // last round's barrier has passed they are copied directly.
             const int S = Ly.stage_rows;
             uint16_t *stK = reinterpret_cast<uint16_t *>(ring);
             uint16_t *stV = stK + (size_t)S * D;
             int32_t *stP = reinterpret_cast<int32_t *>(stV + (size_t)S * D);
             constexpr int LPR = D / 8;  // lanes per row (16 bytes each)
             constexpr int RPW = 32 / LPR;
-            const int R = S * cs;
-            for (int base = 0; count_ok && base < M; base += R) {
-                const int d0 = base + crank * S;
-                const int nd = max(0, min(M - d0, S));
-                for (int j = tid; j < nd; j += kThreads) {
-                    const int dst = d0 + j;
-                    int lo = 0, hi = nwt;  // largest w with gpre[w] <= dst
-                    while (hi - lo > 1) {
-                        const int mid = (lo + hi) >> 1;
-                        if (gpre[mid] <= dst) lo = mid; else hi = mid;
-                    }
-                    const int w = lo;
-                    const int bit = select_bit(gmask[w], dst - gpre[w]);
-                    const int c = w / nwl;
-                    srcidx[j] = min(c * kpc + (w % nwl) * 32 + bit, N - 1);
+            const int wM = M / 32;
+            const int q = count_ok ? gpre[wM] + __popc(gmask[wM] & ((1u << (M % 32)) - 1u)) : 0;
+            // source slot of destination dst: the dst-th kept key
+            auto source_of = [&](int dst) {
+                int lo = 0, hi = nwt;  // largest w with gpre[w] <= dst
+                while (hi - lo > 1) {
+                    const int mid = (lo + hi) >> 1;
+                    if (gpre[mid] <= dst) lo = mid; else hi = mid;
                 }
+                return min(lo * 32 + select_bit(gmask[lo], dst - gpre[lo]), N - 1);
+            };
+            // one round: gather up to S rows into shared memory (all copies in flight at
+            // once), then write them out; hazard rounds put a cluster barrier in between
+            auto round = [&](int d0, int nd, bool hazard) {
+                for (int j = tid; j < nd; j += kThreads) srcidx[j] = source_of(d0 + j);
                 __syncthreads();
+                const int qq = lane % LPR;
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
                     const long long srow = row_of(a, lr, s, g, srcidx[rr]);
-                    const int q = lane % LPR;
-                    cp_async16(stK + (size_t)rr * D + q * 8, a.K + srow * D + q * 8);
-                    cp_async16(stV + (size_t)rr * D + q * 8, a.V + srow * D + q * 8);
-                    if (q == 0) cp_async4(stP + rr, a.pos + srow);
+                    cp_async16(stK + (size_t)rr * D + qq * 8, a.K + srow * D + qq * 8);
+                    cp_async16(stV + (size_t)rr * D + qq * 8, a.V + srow * D + qq * 8);
+                    if (qq == 0) cp_async4(stP + rr, a.pos + srow);
                 }
                 cp_async_wait_all();
                 __syncthreads();
-                cluster.sync();  // every source row of this round is now in shared memory
+                if (hazard) cluster.sync();  // every source row of this round is on chip
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
                     const long long drow = row_of(a, lr, s, g, d0 + rr);
-                    const int q = lane % LPR;
-                    const uint4 xk = *reinterpret_cast<const uint4 *>(stK + (size_t)rr * D + q * 8);
-                    const uint4 xv = *reinterpret_cast<const uint4 *>(stV + (size_t)rr * D + q * 8);
-                    *reinterpret_cast<uint4 *>(a.K + drow * D + q * 8) = xk;
-                    *reinterpret_cast<uint4 *>(a.V + drow * D + q * 8) = xv;
-                    if (q == 0) a.pos[drow] = stP[rr];
+                    const uint4 xk = *reinterpret_cast<const uint4 *>(stK + (size_t)rr * D + qq * 8);
+                    const uint4 xv = *reinterpret_cast<const uint4 *>(stV + (size_t)rr * D + qq * 8);
+                    *reinterpret_cast<uint4 *>(a.K + drow * D + qq * 8) = xk;
+                    *reinterpret_cast<uint4 *>(a.V + drow * D + qq * 8) = xv;
+                    if (qq == 0) a.pos[drow] = stP[rr];
                 }
                 __syncthreads();
+            };
+            const int R = S * cs;
+            for (int base = 0; count_ok && base < q; base += R) {
+                const int d0 = base + crank * S;
+                round(d0, max(0, min(q - d0, S)), true);
             }
+            // rows from slots >= M: no barrier needed once the last hazard round has passed
+            for (int d0 = q + crank * S; count_ok && d0 < M; d0 += R) round(d0, min(M - d0, S), false);
         } else if (a.mode == kModePrune && anyfail_s) {
             if (crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
