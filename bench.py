@@ -283,6 +283,8 @@ def run_ours(args, rank, world, dist_mod):
     if not args.no_e2e and world == 1:
         result["e2e"] = run_e2e(args, cache, ctx, spec, B, restore, stream, keys_rank)
     ctx.close()
+    restore()  # hand back the unpruned cache (the CPU baseline samples it)
+    torch.cuda.synchronize()
     return result, cache, spec
 
 

@@ -170,18 +170,26 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
         if (c->tune_cs > 0 && cs != c->tune_cs) continue;
         const long long kpc = ((long long)(cap_u + cs - 1) / cs + 31) / 32 * 32;
         if (kpc * cs / 32 > 16384) continue;  // global keep mask must fit on chip
+        // buffers per warp: the deepest ring (3 at most) that still leaves room for two
+        // CTAs per SM, else whatever fits one CTA
         int nslot = c->tune_nslot > 0 ? c->tune_nslot : 3;
         tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
         int res = 0;
-        while (nslot >= 1) {
+        for (; nslot >= 1; --nslot) {
             Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
-            if (Ly.total <= budget && Ly.stage_rows >= 16) {
-                res = resident_clusters(c, fn, cs, Ly.total);
-                if (res >= 1 && (c->tune_nslot > 0 || res * cs >= 2 * c->sm_count || nslot == 1)) break;
-                if (res >= 1 && c->tune_nslot > 0) break;
+            if (Ly.total > budget || Ly.stage_rows < 16) {
+                if (c->tune_nslot > 0) break;
+                continue;
             }
-            if (c->tune_nslot > 0) { res = 0; break; }
-            --nslot;
+            int per_sm = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::kThreads, Ly.total) != cudaSuccess) {
+                cudaGetLastError();
+                per_sm = 0;
+            }
+            if (c->tune_nslot > 0 || per_sm >= tri::kMinBlocks || nslot == 1) {
+                res = per_sm >= 1 ? resident_clusters(c, fn, cs, Ly.total) : 0;
+                break;
+            }
         }
         if (res < 1 || nslot < 1) continue;
         Plan p;

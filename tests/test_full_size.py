@@ -1,0 +1,146 @@
+"""Full-size workloads on the GPU, in the launch configuration the benchmark uses.
+
+* Sampled units (first, last, shortest, longest, random) go through the fp64 oracle one by
+  one: raw scores within 1e-4 of each head's scale, kept sets up to threshold ties, compacted
+  rows bit-exact.
+* Every unit is checked without a pristine copy: 64-bit row hashes of K and V (and the
+  positions) are taken before the prune; afterwards slot j of a unit must hold the row of the
+  j-th kept key, the kept set must be exactly the top-B of the kernel's own max-z (ties to the
+  lower slot), and every slot at or beyond min(len, B) must be unchanged.
+"""
+import numpy as np
+import pytest
+import torch
+
+import tri_synth as ts
+import gpu_util as gu
+import oracle
+from rope_aware_key_tri_b200 import tri
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ["qwen3_8b_periodic_36l_3200", "qwen3_8b_oneshot_32k_to_3072", "qwen3_32b_paged_ragged"]
+
+
+def _need_bytes(spec):
+    if spec.lens[0] == "uniform":
+        mean_len = (spec.lens[1] + spec.lens[2]) / 2
+        cap = spec.lens[2]
+    else:
+        mean_len = cap = max(spec.lens)
+    kv = 2 * spec.n_layers * spec.batch * spec.n_kv_heads * mean_len * spec.head_dim * 2
+    zm = spec.n_layers * spec.batch * spec.n_kv_heads * cap * 4
+    return kv * 1.08 + 3 * zm + (8 << 30)
+
+
+def _logical_rows(cache, l):
+    """int64 [batch][Hkv][cap] pool-row index of every logical slot of layer l (-1 = none)."""
+    s = cache.spec
+    cap = cache.cap
+    if not cache.paged:
+        base = ((l * s.batch + torch.arange(s.batch, device="cuda")) * s.n_kv_heads)[:, None] + \
+            torch.arange(s.n_kv_heads, device="cuda")[None, :]
+        return base[:, :, None] * cap + torch.arange(cap, device="cuda")[None, None, :]
+    ps = s.page_size
+    bt = cache.block_table.long()                                   # [batch][max_pages]
+    slot = torch.arange(cap, device="cuda")
+    page = bt[:, slot // ps]                                        # [batch][cap]
+    g = torch.arange(s.n_kv_heads, device="cuda")
+    rows = ((l * cache.n_pages + page[:, None, :]) * s.n_kv_heads + g[None, :, None]) * ps + (slot % ps)
+    return torch.where(page[:, None, :] >= 0, rows, torch.full_like(rows, -1))
+
+
+def _hash_rows(x2d, coeff):
+    return gu.row_hashes(x2d.view(torch.int16), coeff)
+
+
+def _hash_all(flat, coeff, chunk=1 << 20):
+    """Hash of every row of a [rows][d] bf16 view, in chunks (int64 temporaries stay ~1 GB)."""
+    return torch.cat([_hash_rows(flat[i:i + chunk], coeff) for i in range(0, flat.shape[0], chunk)])
+
+
+@pytest.mark.parametrize("name", NAMES)
+def test_full_size_workload(name):
+    spec = ts.WORKLOADS[name]
+    free, _ = torch.cuda.mem_get_info()
+    if _need_bytes(spec) > free:
+        pytest.skip(f"needs {_need_bytes(spec) / 1e9:.0f} GB, {free / 1e9:.0f} GB free")
+    cache = ts.make_cache(spec, seed=2024, device="cuda")
+    torch.cuda.synchronize()
+    s = spec
+    B = s.budget
+    U = cache.n_units
+    lens = cache.lens_host.astype(np.int64)
+    ctx = gu.context_for(cache)
+
+    # ---- sampled units: host copies before anything runs --------------------------------
+    rng = np.random.default_rng(7)
+    seq_short, seq_long = int(np.argmin(lens)), int(np.argmax(lens))
+    picks = {0, U - 1, seq_short * s.n_kv_heads, seq_long * s.n_kv_heads + s.n_kv_heads - 1}
+    picks |= set(int(x) for x in rng.integers(0, U, 2))
+    picks = sorted(picks)
+    rows_in = {u: cache.unit_rows(u) for u in picks}
+    # raw scores of the sampled units' layers (one layer per call, same per-key arithmetic)
+    raw_of = {}
+    for l in sorted(set(cache.unit_index(u)[0] for u in picks)):
+        raw_l, _ = gu.gpu_score(ctx, cache, layer_begin=l, n_layers=1)
+        raw_of[l] = raw_l[0]
+
+    # ---- whole-cache max-z in the launch configuration of the prune ----------------------
+    zmx = torch.full((s.n_layers, s.batch, s.n_kv_heads, cache.cap), float("nan"), device="cuda")
+    ctx.score(cache.K, cache.lens, cache.t, zmax=zmx, block_table=cache.block_table)
+    assert ctx.get_error()[0] == tri.TRI_OK
+
+    # ---- per-row hashes before the prune ---------------------------------------------------
+    gen = torch.Generator(device="cuda").manual_seed(99)
+    coeff = torch.randint(-2**62, 2**62, (s.head_dim,), generator=gen, device="cuda", dtype=torch.int64) | 1
+    flatK = cache.K.view(-1, s.head_dim)
+    flatV = cache.V.view(-1, s.head_dim)
+    hK0 = _hash_all(flatK, coeff)
+    hV0 = _hash_all(flatV, coeff)
+    P0 = cache.pos.clone().view(-1)
+
+    st, code, unit = gu.gpu_prune(ctx, cache)
+    assert st == tri.TRI_OK, (st, code, unit)
+    assert np.array_equal(cache.lens_host, np.minimum(lens, B))
+
+    # ---- sampled units against the oracle ---------------------------------------------------
+    for u in picks:
+        l, b, g = cache.unit_index(u)
+        lab = f"{name} unit {u} (l={l}, s={b}, g={g}, N={lens[b]})"
+        orc = gu.oracle_unit(cache, u, B, rows=rows_in[u])
+        gu.check_scores(raw_of[l][b, g * s.group:(g + 1) * s.group], zmx[l, b, g].cpu().numpy(), orc, lab)
+        out = cache.unit_rows(u)
+        kept = gu.kept_from_output(rows_in[u][2], out[2])
+        gu.check_kept(kept, orc, B, lab)
+        gu.check_compacted(rows_in[u], out, kept, lab)
+
+    # ---- every unit, layer by layer, on the device --------------------------------------
+    hK1 = _hash_all(cache.K.view(-1, s.head_dim), coeff)
+    hV1 = _hash_all(cache.V.view(-1, s.head_dim), coeff)
+    P1 = cache.pos.view(-1)
+    lens_t = torch.as_tensor(lens, device="cuda")
+    slot = torch.arange(cache.cap, device="cuda")
+    for l in range(s.n_layers):
+        rows = _logical_rows(cache, l)                                    # [b][H][cap]
+        valid_rows = rows >= 0
+        r = torch.where(valid_rows, rows, torch.zeros_like(rows))
+        hk0, hv0, p0 = hK0[r], hV0[r], P0[r].long()
+        hk1, hv1 = hK1[r], hV1[r]
+        p1 = P1[r].long()
+        n = lens_t[:, None, None]
+        in_len = slot[None, None, :] < n
+        z = torch.where(in_len, zmx[l], torch.full_like(zmx[l], float("-inf")))
+        order = torch.sort(z, dim=-1, descending=True, stable=True).indices   # ties: lower slot first
+        M = torch.clamp(n, max=B)
+        rank = torch.arange(cache.cap, device="cuda")[None, None, :]
+        take = rank < M                                                   # first M in the order
+        big = torch.full_like(order, cache.cap)
+        kept_sorted = torch.sort(torch.where(take, order, big), dim=-1).values  # ascending kept slots
+        dst = rank < M
+        src = torch.where(dst, kept_sorted, rank)                        # untouched slots map to themselves
+        ok = valid_rows
+        assert torch.equal(torch.where(ok, hk1, 0), torch.where(ok, hk0.gather(-1, src), 0)), f"{name} layer {l}: K rows"
+        assert torch.equal(torch.where(ok, hv1, 0), torch.where(ok, hv0.gather(-1, src), 0)), f"{name} layer {l}: V rows"
+        assert torch.equal(torch.where(ok, p1, 0), torch.where(ok, p0.gather(-1, src), 0)), f"{name} layer {l}: positions"
+    ctx.close()
