@@ -958,12 +958,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
             // round's sources into shared memory, the cluster synchronises, then all write.
             // The other M - q kept rows come from slots >= M, which no write touches; once the
             // last round's barrier has passed they are copied directly.
-            const int S = Ly.stage_rows;
-            uint16_t *stK = reinterpret_cast<uint16_t *>(ring);
-            uint16_t *stV = stK + (size_t)S * D;
-            int32_t *stP = reinterpret_cast<int32_t *>(stV + (size_t)S * D);
+            // Two staging buffers in the (idle) TMA ring: the sources of round r + 1 are
+            // fetched while round r is written out. Round r + 1 reads slots >= its own
+            // destinations, all above the destinations of round r, so the overlap is safe.
             constexpr int LPR = D / 8;  // lanes per row (16 bytes each)
             constexpr int RPW = 32 / LPR;
+            const unsigned ring_bytes = (unsigned)kWarps * nslot * kStageBytes;
+            const int S2 = (int)((ring_bytes / 2u) / (unsigned)(4 * D + 4)) / 16 * 16;
+            const unsigned buf_bytes = (unsigned)S2 * (4 * D + 4);
             const int wM = M / 32;
             const int q = count_ok ? gpre[wM] + __popc(gmask[wM] & ((1u << (M % 32)) - 1u)) : 0;
             // source slot of destination dst: the dst-th kept key
@@ -975,21 +977,57 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 }
                 return min(lo * 32 + select_bit(gmask[lo], dst - gpre[lo]), N - 1);
             };
-            // one round: gather up to S rows into shared memory (all copies in flight at
-            // once), then write them out; hazard rounds put a cluster barrier in between
-            auto round = [&](int d0, int nd, bool hazard) {
-                for (int j = tid; j < nd; j += kThreads) srcidx[j] = source_of(d0 + j);
+            const int R = S2 * cs;
+            const int H = count_ok ? (q + R - 1) / R : 0;                    // hazard rounds
+            const int dfirst = q + crank * S2;
+            const int Dk = (count_ok && dfirst < M) ? (M - dfirst + R - 1) / R : 0;  // direct rounds
+            const int NR = H + Dk;
+            auto round_span = [&](int r, int &nd) {
+                int d0;
+                if (r < H) {
+                    d0 = r * R + crank * S2;
+                    nd = max(0, min(q - d0, S2));
+                } else {
+                    d0 = dfirst + (r - H) * R;
+                    nd = max(0, min(M - d0, S2));
+                }
+                return d0;
+            };
+            const int qq = lane % LPR;
+            auto fetch = [&](int r) {
+                int nd;
+                const int d0 = round_span(r, nd);
+                unsigned char *buf = ring + (r & 1) * buf_bytes;
+                uint16_t *stK = reinterpret_cast<uint16_t *>(buf);
+                uint16_t *stV = stK + (size_t)S2 * D;
+                int32_t *stP = reinterpret_cast<int32_t *>(stV + (size_t)S2 * D);
+                int *sidx = srcidx + (r & 1) * S2;
+                for (int j = tid; j < nd; j += kThreads) sidx[j] = source_of(d0 + j);
                 __syncthreads();
-                const int qq = lane % LPR;
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
-                    const long long srow = row_of(a, lr, s, g, srcidx[rr]);
+                    const long long srow = row_of(a, lr, s, g, sidx[rr]);
                     cp_async16(stK + (size_t)rr * D + qq * 8, a.K + srow * D + qq * 8);
                     cp_async16(stV + (size_t)rr * D + qq * 8, a.V + srow * D + qq * 8);
                     if (qq == 0) cp_async4(stP + rr, a.pos + srow);
                 }
-                cp_async_wait_all();
+                asm volatile("cp.async.commit_group;" ::: "memory");
+            };
+            if (NR > 0) fetch(0);
+            for (int r = 0; r < NR; ++r) {
+                if (r + 1 < NR) {
+                    fetch(r + 1);
+                    asm volatile("cp.async.wait_group 1;" ::: "memory");
+                } else {
+                    asm volatile("cp.async.wait_group 0;" ::: "memory");
+                }
                 __syncthreads();
-                if (hazard) cluster.sync();  // every source row of this round is on chip
+                if (r < H) cluster.sync();  // every source row of this hazard round is on chip
+                int nd;
+                const int d0 = round_span(r, nd);
+                const unsigned char *buf = ring + (r & 1) * buf_bytes;
+                const uint16_t *stK = reinterpret_cast<const uint16_t *>(buf);
+                const uint16_t *stV = stK + (size_t)S2 * D;
+                const int32_t *stP = reinterpret_cast<const int32_t *>(stV + (size_t)S2 * D);
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
                     const long long drow = row_of(a, lr, s, g, d0 + rr);
                     const uint4 xk = *reinterpret_cast<const uint4 *>(stK + (size_t)rr * D + qq * 8);
@@ -999,14 +1037,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                     if (qq == 0) a.pos[drow] = stP[rr];
                 }
                 __syncthreads();
-            };
-            const int R = S * cs;
-            for (int base = 0; count_ok && base < q; base += R) {
-                const int d0 = base + crank * S;
-                round(d0, max(0, min(q - d0, S)), true);
             }
-            // rows from slots >= M: no barrier needed once the last hazard round has passed
-            for (int d0 = q + crank * S; count_ok && d0 < M; d0 += R) round(d0, min(M - d0, S), false);
         } else if (a.mode == kModePrune && anyfail_s) {
             if (crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
