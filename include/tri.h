@@ -155,6 +155,29 @@ TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads
 TRI_API tri_status tri_prune(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream);
 
 /*
+ * tri_prune without any device allocation at call time. (The TriAttention pages have no
+ * counterpart: this is an interface for callers that cannot allocate device memory while they
+ * run, e.g. a serving loop whose device memory belongs to another allocator, or one that cannot
+ * afford the device-wide synchronisation of the cudaFree that tri_prune performs when it grows
+ * its scratch.)
+ *   Same arguments, semantics and results as tri_prune. The scores of the units in flight live
+ *   in a fixed 64 MiB device array that the library holds on every GPU that loads it, until the
+ *   process exits; sequences the device refuses are flagged in a fixed array of 16384 entries.
+ *   It calls no cudaMalloc or cudaFree; it zeroes the flags with cudaMemsetAsync on `stream`.
+ * Limits: batch <= 16384; the unit-capacity limit of tri_prune applies unchanged (within it
+ *   one unit's score slot, capacity * (group + 1) floats, stays below 19 MB). When the 64 MiB
+ *   holds fewer slots than tri_prune would run clusters, fewer clusters run: same results, a
+ *   longer run. Sizes beyond the limits return TRI_EUNSUPPORTED and tri_last_error says why;
+ *   nothing is launched.
+ * The first call on a device looks up the arrays' device addresses (cudaGetSymbolAddress);
+ *   make that first call before any stream capture. Every call shares the two arrays and
+ *   leaves its contents there: calls that overlap on the GPU (other streams, other contexts on
+ *   the same device) race on them and must be serialised by the caller.
+ */
+TRI_API tri_status tri_prune_noalloc(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, int32_t budget,
+                                     void *stream);
+
+/*
  * Debug / parity entry: score without pruning.
  *   raw   float [n_layers][batch][n_kv_heads*group][cap_u] or NULL: s_h(i) per query head
  *   zmax  float [n_layers][batch][n_kv_heads][cap_u] or NULL: max over the group of z_h(i)

@@ -327,6 +327,173 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     return TRI_OK;
 }
 
+// ---------------------------------------------------------------------------------------
+// Allocation-free prune. Some callers cannot allocate device memory at call time: a serving
+// loop whose device memory is owned by another allocator, or one that cannot afford the
+// device-wide synchronisation that cudaFree implies when tri_prune has to grow its scratch.
+// For them the per-cluster score slots (and the per-sequence refusal flags) live in
+// file-scope device arrays of fixed size, loaded with the library and held until exit.
+// ---------------------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // score slots: 64 MiB
+constexpr int kNoAllocMaxBatch = 16384;                       // refusal flags
+constexpr int kMaxDevices = 64;
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];
+static __device__ __align__(256) int32_t g_noalloc_seq_bad[kNoAllocMaxBatch];
+
+struct NoAllocSymbols {
+    bool ready = false;
+    float *scratch = nullptr;
+    int32_t *seq_bad = nullptr;
+};
+std::mutex g_noalloc_mu;
+NoAllocSymbols g_noalloc[kMaxDevices];
+
+// Device addresses of the two arrays on the context's device (set up once per device, with
+// that device current). The host-side names are stand-ins, never device addresses.
+tri_status noalloc_symbols(tri_ctx *c, NoAllocSymbols *out) {
+    if (c->device < 0 || c->device >= kMaxDevices) return TRI_EUNSUPPORTED;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    NoAllocSymbols &e = g_noalloc[c->device];
+    if (!e.ready) {
+        cudaError_t ce = cudaSetDevice(c->device);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+        void *p = nullptr;
+        ce = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaGetSymbolAddress(g_noalloc_scratch)");
+        e.scratch = static_cast<float *>(p);
+        p = nullptr;
+        ce = cudaGetSymbolAddress(&p, g_noalloc_seq_bad);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaGetSymbolAddress(g_noalloc_seq_bad)");
+        e.seq_bad = static_cast<int32_t *>(p);
+        e.ready = true;
+    }
+    *out = e;
+    return TRI_OK;
+}
+
+tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
+    if (!c || !kv || !t) return TRI_EINVAL;
+    if (!c->loaded) return TRI_ESTATE;
+    if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
+        return TRI_EINVAL;
+    const bool paged = kv->block_table != nullptr;
+    long long cap_u;
+    if (paged) {
+        if (kv->page_size < 16 || kv->page_size % 16 != 0 || kv->max_pages < 1 || kv->n_pages < 1)
+            return TRI_EINVAL;
+        cap_u = (long long)kv->page_size * kv->max_pages;
+    } else {
+        if (kv->cap < 1) return TRI_EINVAL;
+        cap_u = kv->cap;
+    }
+    if (cap_u > (1LL << 30)) return TRI_EUNSUPPORTED;
+    if (budget < 1) return TRI_EINVAL;
+    if (!kv->K || !kv->V || !kv->pos || !kv->lens) return TRI_EINVAL;
+    if (!aligned(kv->K, 16) || !aligned(kv->V, 16) || !aligned(kv->pos, 4)) return TRI_EINVAL;
+    if (!is_device_ptr(kv->K) || !is_device_ptr(kv->V) || !is_device_ptr(kv->pos)) return TRI_EINVAL;
+    if (kv->lens_out && (!is_device_ptr(kv->lens_out) || !aligned(kv->lens_out, 4))) return TRI_EINVAL;
+    if (!is_device_ptr(kv->lens) || !is_device_ptr(t) || !aligned(kv->lens, 4) || !aligned(t, 4))
+        return TRI_EINVAL;
+    if (paged && (!is_device_ptr(kv->block_table) || !aligned(kv->block_table, 4))) return TRI_EINVAL;
+    if (kv->batch > kNoAllocMaxBatch) {
+        std::snprintf(c->last_error, sizeof c->last_error,
+                      "tri_prune_noalloc: batch %d exceeds the fixed flag array (%d sequences)", kv->batch,
+                      kNoAllocMaxBatch);
+        return TRI_EUNSUPPORTED;
+    }
+    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
+    if (n_units * tri::kMaxCluster > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+
+    KernelFn fn = pick_kernel(c->D, c->G, c->layout);
+    if (!fn) return TRI_EUNSUPPORTED;
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+    NoAllocSymbols sym;
+    tri_status st = noalloc_symbols(c, &sym);
+    if (st != TRI_OK) return st;
+    ce = prepare_kernel(fn, c->max_smem_optin);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute");
+    Plan plan;
+    st = plan_launch(c, fn, (int)cap_u, n_units, &plan);
+    if (st == TRI_EUNSUPPORTED) {
+        std::snprintf(c->last_error, sizeof c->last_error,
+                      "tri_prune_noalloc: no launch shape holds a unit capacity of %lld slots on chip", cap_u);
+        return st;
+    }
+    if (st != TRI_OK) return st;
+
+    // as many resident clusters as the fixed scratch holds slots for (the grid is persistent,
+    // so fewer clusters still cover every unit)
+    const long long slot_floats = ((long long)cap_u * (c->G + 1) + 31) / 32 * 32;
+    const long long slots = (long long)(kNoAllocScratchBytes / sizeof(float)) / slot_floats;
+    if (slots < 1) {
+        std::snprintf(c->last_error, sizeof c->last_error,
+                      "tri_prune_noalloc: a unit of %lld slots needs %lld bytes of scratch, above the fixed "
+                      "%zu bytes (at most %lld slots per unit for this group size)",
+                      cap_u, slot_floats * 4, kNoAllocScratchBytes,
+                      (long long)(kNoAllocScratchBytes / sizeof(float)) / (c->G + 1) / 32 * 32);
+        return TRI_EUNSUPPORTED;
+    }
+    const int n_clusters = (int)std::min<long long>(plan.n_clusters, slots);
+
+    const bool finalize = kv->lens_out != nullptr;
+    if (finalize) {
+        // the refusal flags must start at zero; they keep whatever the last call left
+        ce = cudaMemsetAsync(sym.seq_bad, 0, sizeof(int32_t) * kv->batch, static_cast<cudaStream_t>(stream));
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaMemsetAsync(flags)");
+    }
+
+    tri::Args a;
+    std::memset(&a, 0, sizeof a);
+    a.K = static_cast<uint16_t *>(kv->K);
+    a.V = static_cast<uint16_t *>(kv->V);
+    a.pos = kv->pos;
+    a.lens = kv->lens;
+    a.lens_out = finalize ? kv->lens_out : nullptr;
+    a.block_table = kv->block_table;
+    a.t = t;
+    a.batch = kv->batch;
+    a.n_kv = c->Hkv;
+    a.cap_u = (int)cap_u;
+    a.paged = paged ? 1 : 0;
+    a.page_size = paged ? kv->page_size : 0;
+    a.max_pages = paged ? kv->max_pages : 0;
+    a.n_pages = paged ? kv->n_pages : 0;
+    a.layer_begin = kv->layer_begin;
+    a.budget = budget;
+    a.omega = c->d_omega;
+    a.Qc = c->d_Qc;
+    a.w = c->d_w;
+    a.mode = tri::kModePrune;
+    a.cs = plan.cs;
+    a.kpc_max = plan.kpc;
+    a.nslot = plan.nslot;
+    a.n_units = (int)n_units;
+    a.scratch = sym.scratch;
+    a.slot_floats = slot_floats;
+    a.status = c->d_status;
+    a.counter = c->d_counter;
+    a.seq_bad = finalize ? sym.seq_bad : nullptr;
+
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)(n_clusters * plan.cs));
+    cfg.blockDim = dim3(tri::kThreads);
+    cfg.dynamicSmemBytes = plan.smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)plan.cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    ce = cudaLaunchKernelEx(&cfg, fn, a);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx");
+    return TRI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -441,6 +608,10 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
 
 tri_status tri_prune(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
     return run(c, kv, t, budget, nullptr, nullptr, tri::kModePrune, stream);
+}
+
+tri_status tri_prune_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
+    return run_noalloc(c, kv, t, budget, stream);
 }
 
 tri_status tri_score(tri_ctx *c, const tri_kv *kv, const int32_t *t, float *raw, float *zmax, void *stream) {

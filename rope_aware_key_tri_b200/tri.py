@@ -60,6 +60,7 @@ def _load():
     L.tri_calibrate_load.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, D,
                                      ctypes.c_int, P, P, P, P, ctypes.c_int]
     L.tri_prune.argtypes = [P, ctypes.POINTER(tri_kv), P, I32, P]
+    L.tri_prune_noalloc.argtypes = [P, ctypes.POINTER(tri_kv), P, I32, P]
     L.tri_score.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
     L.tri_set_tuning.argtypes = [P, ctypes.c_int, ctypes.c_int]
@@ -67,7 +68,7 @@ def _load():
     L.tri_last_error.restype = ctypes.c_char_p
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
-    for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_score",
+    for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
                "tri_get_error", "tri_set_tuning", "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
     return L
@@ -119,6 +120,10 @@ def tri_calibrate_load(ctx, n_layers, n_kv_heads, group, head_dim, rope_base, la
 
 def tri_prune(ctx, kv: tri_kv, t_ptr: int, budget: int, stream: int) -> int:
     return _lib.tri_prune(ctx, ctypes.byref(kv), t_ptr, int(budget), stream)
+
+
+def tri_prune_noalloc(ctx, kv: tri_kv, t_ptr: int, budget: int, stream: int) -> int:
+    return _lib.tri_prune_noalloc(ctx, ctypes.byref(kv), t_ptr, int(budget), stream)
 
 
 def tri_score(ctx, kv: tri_kv, t_ptr: int, raw_ptr: int, zmax_ptr: int, stream: int) -> int:
@@ -222,6 +227,17 @@ class TriContext:
         st = tri_prune(self.handle, kv, t.data_ptr(), budget, _stream_handle(stream))
         if check and st != TRI_OK:
             raise TriError(st, "tri_prune", tri_last_error(self.handle))
+        return st
+
+    def prune_noalloc(self, K, V, pos, lens, t, budget, lens_out="inplace", block_table=None,
+                      layer_begin=0, stream=None, check=True):
+        """tri_prune_noalloc: the same prune with fixed, library-held scratch (no allocation)."""
+        if isinstance(lens_out, str):
+            lens_out = lens
+        kv = make_kv(K, V, pos, lens, lens_out, block_table, layer_begin=layer_begin)
+        st = tri_prune_noalloc(self.handle, kv, t.data_ptr(), budget, _stream_handle(stream))
+        if check and st != TRI_OK:
+            raise TriError(st, "tri_prune_noalloc", tri_last_error(self.handle))
         return st
 
     def score(self, K, lens, t, raw=None, zmax=None, block_table=None, layer_begin=0,
