@@ -787,28 +787,45 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
                 __syncwarp();
             }
-            const int lim = (n_local + 31) / 32 * 32;
-#pragma unroll 4
-            for (int i = tid; i < lim; i += kThreads) {
-                const bool in = i < n_local;
-                unsigned key = 0u;
-                if (in) {
-                    float sv[G];
-                    load_scores<G>(sc_local + i * G, sv);
-                    float z = -__int_as_float(0x7f800000);
+            float mu_r[G], is_r[G];
 #pragma unroll
-                    for (int h = 0; h < G; ++h) z = fmaxf(z, (sv[h] - muf_s[h]) * inv_s[h]);
-                    z = z + 0.0f;  // -0 -> +0
-                    if (zrow) zrow[i] = z;
-                    key = float_key(z);
-                    uk[i] = key;
+            for (int h = 0; h < G; ++h) {
+                mu_r[h] = muf_s[h];
+                is_r[h] = inv_s[h];
+            }
+            // the scores come back from L2 in batches: every load of a batch is in flight
+            // before the first one is used
+            constexpr int ZB = (G >= 8 && LAYOUT == 1) ? 1 : ((G >= 8 || LAYOUT == 1) ? 2 : 4);
+            const int lim = (n_local + 31) / 32 * 32;
+            for (int base = warp * 32; base < lim; base += ZB * kThreads) {
+                float sv[ZB][G];
+#pragma unroll
+                for (int k = 0; k < ZB; ++k) {
+                    const int i = base + k * kThreads + lane;
+                    if (i < n_local) load_scores<G>(sc_local + i * G, sv[k]);
                 }
-                if (selecting) {
-                    const unsigned bin = key >> 24;
-                    const unsigned act = __ballot_sync(FULL, in);
+#pragma unroll
+                for (int k = 0; k < ZB; ++k) {
+                    if (base + k * kThreads >= lim) break;  // uniform over the warp
+                    const int i = base + k * kThreads + lane;
+                    const bool in = i < n_local;
+                    unsigned key = 0u;
                     if (in) {
-                        const unsigned peers = __match_any_sync(act, bin);
-                        if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
+                        float z = -__int_as_float(0x7f800000);
+#pragma unroll
+                        for (int h = 0; h < G; ++h) z = fmaxf(z, (sv[k][h] - mu_r[h]) * is_r[h]);
+                        z = z + 0.0f;  // -0 -> +0
+                        if (zrow) zrow[i] = z;
+                        key = float_key(z);
+                        uk[i] = key;
+                    }
+                    if (selecting) {
+                        const unsigned bin = key >> 24;
+                        const unsigned act = __ballot_sync(FULL, in);
+                        if (in) {
+                            const unsigned peers = __match_any_sync(act, bin);
+                            if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
+                        }
                     }
                 }
             }
