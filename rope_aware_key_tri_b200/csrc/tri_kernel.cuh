@@ -587,9 +587,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 cw[i][p] = make_float2(coef_w[hq * F + b0], coef_w[hq * F + b0 + 1]);
             }
         }
-        float *raw_row = nullptr;
-        if (a.raw)
-            raw_row = a.raw + (((long long)lr * a.batch + s) * Hq + (long long)g * G + hx) * (long long)a.cap_u + begin;
         float *sc_local = sc + (long long)begin * G;
 
         // ---- score loop ----------------------------------------------------------------
@@ -618,7 +615,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
             const uint16_t *lane_a = stage + kw * D + sub * DH;
             const int li0 = st * kStageRows + kw;
             float *sc_pass = sc_local + li0 * G + hx;
-            float *raw_pass = raw_row ? raw_row + li0 : nullptr;
             const int valid = n_local - li0;  // key of pass p is valid when p * KPP < valid
 #pragma unroll
             for (int pass = 0; pass < kStageRows / KPP; ++pass) {
@@ -676,7 +672,6 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 }
                 if (writer && pass * KPP < valid) {
                     st_hint(sc_pass + pass * KPP * G, v[0], pol_last);
-                    if (raw_pass) raw_pass[pass * KPP] = v[0];
                     const double dv = (double)v[0];
                     m_s += dv;
                     m_q = fma(dv, dv, m_q);
@@ -778,6 +773,10 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
         // slot; the first radix digit's histogram is built on the way.
         float *zrow = a.zmax ? a.zmax + (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + begin
                              : nullptr;
+        // raw scores, when asked for, are copied out here from the values read back (the
+        // scoring loop stays free of the extra stores)
+        float *raw_row = a.raw ? a.raw + (((long long)lr * a.batch + s) * Hq + (long long)g * G) * (long long)a.cap_u + begin
+                               : nullptr;
         const bool keys_on_chip = (long long)n_local * 4 <= (long long)kWarps * nslot * kStageBytes;
         unsigned *uk = keys_on_chip ? reinterpret_cast<unsigned *>(ring) : ukey + begin;
         const bool selecting = a.mode == kModePrune && !anyfail_s;
@@ -816,17 +815,14 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                         for (int h = 0; h < G; ++h) z = fmaxf(z, (sv[k][h] - mu_r[h]) * is_r[h]);
                         z = z + 0.0f;  // -0 -> +0
                         if (zrow) zrow[i] = z;
+                        if (raw_row) {
+#pragma unroll
+                            for (int h = 0; h < G; ++h) raw_row[(long long)h * a.cap_u + i] = sv[k][h];
+                        }
                         key = float_key(z);
                         uk[i] = key;
                     }
-                    if (selecting) {
-                        const unsigned bin = key >> 24;
-                        const unsigned act = __ballot_sync(FULL, in);
-                        if (in) {
-                            const unsigned peers = __match_any_sync(act, bin);
-                            if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
-                        }
-                    }
+                    if (selecting && in) atomicAdd(wh + (key >> 24), 1u);
                 }
             }
         }
@@ -840,21 +836,17 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
             for (int pass = 0; pass < 4 && !resolved; ++pass) {
                 const int shift = 24 - 8 * pass;
                 unsigned *wh = whist + warp * kBins;
-                const int lim = pass == 0 ? 0 : (n_local + 31) / 32 * 32;  // pass 0 built above
+                const int lim = pass == 0 ? 0 : n_local;  // pass 0 built above
                 if (pass > 0) {
                     for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
                     __syncwarp();
                 }
+                // after the first digit few keys still match the prefix, and those spread over
+                // the bins: plain shared-memory atomics, no warp-level aggregation
+#pragma unroll 4
                 for (int i = tid; i < lim; i += kThreads) {
-                    const bool in = i < n_local;
-                    const unsigned u = in ? uk[i] : 0u;
-                    const bool m = in && ((u & pmask) == prefix);
-                    const unsigned bin = (u >> shift) & 255u;
-                    const unsigned act = __ballot_sync(FULL, m);
-                    if (m) {
-                        const unsigned peers = __match_any_sync(act, bin);
-                        if (lane == __ffs(peers) - 1) atomicAdd(wh + bin, (unsigned)__popc(peers));
-                    }
+                    const unsigned u = uk[i];
+                    if ((u & pmask) == prefix) atomicAdd(wh + ((u >> shift) & 255u), 1u);
                 }
                 __syncthreads();
                 unsigned *bh = bhist + (pass & 1) * kBins;
