@@ -42,6 +42,15 @@ struct tri_ctx {
     int tune_nslot = 0;
     // text of the last failure seen on the host (CUDA error name and the call that failed)
     char last_error[256] = {0};
+    // the last launch shape planned, reused while the call shape and tuning repeat
+    struct {
+        bool valid = false;
+        const void *fn = nullptr;
+        long long cap_u = 0, n_units = 0;
+        int tune_cs = 0, tune_nslot = 0;
+        int cs = 0, nslot = 0, kpc = 0, n_clusters = 0, extra = 0;
+        size_t smem = 0;
+    } plan_cache;
 };
 
 namespace {
@@ -103,7 +112,7 @@ tri_status cuda_fail(tri_ctx *c, cudaError_t e, const char *what, tri_status st 
 }
 
 struct Plan {
-    int cs = 0, nslot = 0, kpc = 0, n_clusters = 0;
+    int cs = 0, nslot = 0, kpc = 0, n_clusters = 0, extra = 0;
     size_t smem = 0;
 };
 
@@ -136,7 +145,7 @@ int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem) {
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)cs);
-    cfg.blockDim = dim3(tri::kThreads);
+    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -160,6 +169,17 @@ int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem) {
 // live score slots (one per resident cluster) within the L2 budget; if none does both,
 // the largest cs that fits.
 tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Plan *out) {
+    auto &pc = c->plan_cache;
+    if (pc.valid && pc.fn == (const void *)fn && pc.cap_u == cap_u && pc.n_units == n_units &&
+        pc.tune_cs == c->tune_cs && pc.tune_nslot == c->tune_nslot) {
+        out->cs = pc.cs;
+        out->nslot = pc.nslot;
+        out->kpc = pc.kpc;
+        out->n_clusters = pc.n_clusters;
+        out->extra = pc.extra;
+        out->smem = pc.smem;
+        return TRI_OK;
+    }
     cudaFuncAttributes fa;
     cudaError_t fe = cudaFuncGetAttributes(&fa, fn);
     if (fe != cudaSuccess) return cuda_fail(c, fe, "cudaFuncGetAttributes");
@@ -173,16 +193,16 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
         // buffers per warp: the deepest ring (3 at most) that still leaves room for two
         // CTAs per SM, else whatever fits one CTA
         int nslot = c->tune_nslot > 0 ? c->tune_nslot : 3;
-        tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
+        tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0);
         int res = 0;
         for (; nslot >= 1; --nslot) {
-            Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs);
+            Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0);
             if (Ly.total > budget || Ly.stage_rows < 16) {
                 if (c->tune_nslot > 0) break;
                 continue;
             }
             int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::kThreads, Ly.total) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::cta_threads(c->G), Ly.total) != cudaSuccess) {
                 cudaGetLastError();
                 per_sm = 0;
             }
@@ -192,7 +212,31 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
             }
         }
         if (res < 1 || nslot < 1) continue;
+        // shared memory left over at this occupancy goes to the compaction's staging
+        int extra = 0;
+        for (int e = 64 * 1024; e >= 8 * 1024; e -= 8 * 1024) {
+            const tri::Layout Le = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, e);
+            if (Le.total > budget) continue;
+            int per_sm_e = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_e, fn, tri::cta_threads(c->G), Le.total) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                continue;
+            }
+            int per_sm0 = 0;
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm0, fn, tri::cta_threads(c->G), Ly.total) !=
+                cudaSuccess) {
+                cudaGetLastError();
+                break;
+            }
+            if (per_sm_e >= per_sm0) {
+                extra = e;
+                Ly = Le;
+                break;
+            }
+        }
         Plan p;
+        p.extra = extra;
         p.cs = cs;
         p.nslot = nslot;
         p.kpc = (int)kpc;
@@ -205,6 +249,18 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
     }
     if (best.cs == 0) return TRI_EUNSUPPORTED;
     *out = best;
+    pc.valid = true;
+    pc.fn = (const void *)fn;
+    pc.cap_u = cap_u;
+    pc.n_units = n_units;
+    pc.tune_cs = c->tune_cs;
+    pc.tune_nslot = c->tune_nslot;
+    pc.cs = best.cs;
+    pc.nslot = best.nslot;
+    pc.kpc = best.kpc;
+    pc.n_clusters = best.n_clusters;
+    pc.extra = best.extra;
+    pc.smem = best.smem;
     return TRI_OK;
 }
 
@@ -302,6 +358,7 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     a.cs = plan.cs;
     a.kpc_max = plan.kpc;
     a.nslot = plan.nslot;
+    a.ring_extra = plan.extra;
     a.n_units = (int)n_units;
     a.scratch = c->d_scratch;
     a.slot_floats = slot_floats;
@@ -312,7 +369,7 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)(plan.n_clusters * plan.cs));
-    cfg.blockDim = dim3(tri::kThreads);
+    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
@@ -469,6 +526,7 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     a.cs = plan.cs;
     a.kpc_max = plan.kpc;
     a.nslot = plan.nslot;
+    a.ring_extra = plan.extra;
     a.n_units = (int)n_units;
     a.scratch = sym.scratch;
     a.slot_floats = slot_floats;
@@ -479,7 +537,7 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)(n_clusters * plan.cs));
-    cfg.blockDim = dim3(tri::kThreads);
+    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];

@@ -49,8 +49,11 @@ namespace cg = cooperative_groups;
 
 constexpr int kStageRows = 16;      // rows per TMA bulk copy (one copy never crosses a page)
 constexpr int kBins = 256;          // radix digit width: 8 bits
-constexpr int kWarps = 6;           // warps per CTA (two CTAs per SM)
-constexpr int kThreads = kWarps * 32;
+// Warps per CTA (two CTAs per SM). A lane keeps 48 coefficients in registers with 8 warps
+// (128 registers per thread) and 96 with 6 warps (168); GQA 8 needs the latter.
+__host__ __device__ constexpr int cta_warps(int G) { return G >= 8 ? 6 : 8; }
+__host__ __device__ constexpr int cta_threads(int G) { return cta_warps(G) * 32; }
+constexpr int kMaxWarps = 8;
 constexpr int kMinBlocks = 2;
 constexpr int kMaxCluster = 16;
 constexpr int kModePrune = 0;
@@ -83,6 +86,7 @@ struct Args {
     int mode;
     int cs;                      // cluster size (CTAs per unit)
     int kpc_max;                 // key capacity of one CTA (multiple of 32)
+    int ring_extra;              // staging bytes appended to the TMA ring
     int nslot;                   // TMA buffers per warp
     float *scratch;              // per-cluster slots: [cap_u][G] scores then [cap_u] order keys
     long long slot_floats;       // floats per slot
@@ -107,17 +111,22 @@ struct Layout {
     unsigned ring, coef_t, coef_w, phase, whist, bhist, ghist, lmask, gmask, gpre, xch, misc,
         srcidx, bars, total;
     int stage_rows;    // compaction rows per CTA per round (staged in the ring)
+    unsigned ring_bytes;  // the TMA ring plus the extra staging the compaction may use
 };
 
 __host__ __device__ inline unsigned align_up(unsigned x, unsigned a) { return (x + a - 1) / a * a; }
 
-__host__ __device__ inline Layout make_layout(int D, int G, int nslot, int kpc, int cs) {
+// extra: bytes appended to the TMA ring where shared memory is left over; the order keys and
+// the compaction's staging use the whole region, the key stream only the ring.
+__host__ __device__ inline Layout make_layout(int D, int G, int nslot, int kpc, int cs, int extra) {
+    const int kWarps = cta_warps(G);
     Layout L;
     unsigned o = 0;
     const int F = D / 2;
     const int nwl = kpc / 32;
     L.ring = o;
-    o = align_up(o + (unsigned)kWarps * nslot * kStageRows * D * 2u, 128);
+    o = align_up(o + (unsigned)kWarps * nslot * kStageRows * D * 2u + (unsigned)extra, 128);
+    L.ring_bytes = o;
     const unsigned row_bytes = (unsigned)D * 2u * 2u + 4u;
     int S = (int)(o / row_bytes);
     S = S / 16 * 16;
@@ -289,7 +298,9 @@ __device__ __forceinline__ int select_bit(unsigned m, int k) {
 
 // Exclusive scan of n ints in place in shared memory (any n); returns the total.
 // All threads of the block must call it.
+template <int kWarps>
 __device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 ints */) {
+    constexpr int kThreads = kWarps * 32;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     constexpr int PER = 4;
     int carry = 0;
@@ -337,12 +348,12 @@ __device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 in
 // Per-key slice geometry. A key of D dims is split over LPK lanes; each lane holds DH
 // consecutive dims from the first half of the row and the DH dims D/2 further on, i.e.
 // DH whole bands in either rotary layout. DH is chosen so that a lane keeps 3 * DH * G
-// (= 96) coefficients in registers: its DH trig coefficients of each half and its DH
+// (48 with 8 warps, 96 with 6) coefficients in registers: its DH trig coefficients of each half and its DH
 // norm weights, for every head of the group.
 // ---------------------------------------------------------------------------------
 template <int D, int G>
 struct Geo {
-    static constexpr int DH_REG = G == 8 ? 4 : (G == 4 ? 8 : (G == 2 ? 16 : 32));
+    static constexpr int DH_REG = (cta_warps(G) == 8 ? 16 : 32) / G;
     static constexpr int DH = DH_REG < D / 4 ? DH_REG : D / 4;  // at least 2 lanes per key
     static constexpr int LPK = D / (2 * DH);
     static constexpr int KPP = 32 / LPK;  // keys per warp per pass
@@ -412,7 +423,9 @@ __host__ __device__ constexpr int pair_dim(int p, int e) {
 // The fused kernel. Grid: n_clusters * cs CTAs (clusters of cs), persistent over units.
 // ---------------------------------------------------------------------------------
 template <int D, int G, int LAYOUT>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const Args a) {
+__global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(const Args a) {
+    constexpr int kWarps = cta_warps(G);
+    constexpr int kThreads = kWarps * 32;
     constexpr int F = D / 2;
     using GE = Geo<D, G>;
     constexpr int DH = GE::DH;
@@ -430,7 +443,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
     const int n_clusters = gridDim.x / cs;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nslot = a.nslot;
-    const Layout Ly = make_layout(D, G, nslot, a.kpc_max, cs);
+    const Layout Ly = make_layout(D, G, nslot, a.kpc_max, cs, a.ring_extra);
 
     unsigned char *ring = smem + Ly.ring;
     float *coef_t = reinterpret_cast<float *>(smem + Ly.coef_t);
@@ -777,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
         // scoring loop stays free of the extra stores)
         float *raw_row = a.raw ? a.raw + (((long long)lr * a.batch + s) * Hq + (long long)g * G) * (long long)a.cap_u + begin
                                : nullptr;
-        const bool keys_on_chip = (long long)n_local * 4 <= (long long)kWarps * nslot * kStageBytes;
+        const bool keys_on_chip = (long long)n_local * 4 <= (long long)Ly.ring_bytes;
         unsigned *uk = keys_on_chip ? reinterpret_cast<unsigned *>(ring) : ukey + begin;
         const bool selecting = a.mode == kModePrune && !anyfail_s;
         {
@@ -795,34 +808,34 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
             // the scores come back from L2 in batches: every load of a batch is in flight
             // before the first one is used
             constexpr int ZB = (G >= 8 && LAYOUT == 1) ? 1 : ((G >= 8 || LAYOUT == 1) ? 2 : 4);
-            const int lim = (n_local + 31) / 32 * 32;
-            for (int base = warp * 32; base < lim; base += ZB * kThreads) {
+            for (int base = tid; base < n_local; base += ZB * kThreads) {
                 float sv[ZB][G];
 #pragma unroll
                 for (int k = 0; k < ZB; ++k) {
-                    const int i = base + k * kThreads + lane;
+                    const int i = base + k * kThreads;
                     if (i < n_local) load_scores<G>(sc_local + i * G, sv[k]);
                 }
 #pragma unroll
                 for (int k = 0; k < ZB; ++k) {
-                    if (base + k * kThreads >= lim) break;  // uniform over the warp
-                    const int i = base + k * kThreads + lane;
-                    const bool in = i < n_local;
-                    unsigned key = 0u;
-                    if (in) {
+                    const int i = base + k * kThreads;
+                    if (i < n_local) {
                         float z = -__int_as_float(0x7f800000);
 #pragma unroll
                         for (int h = 0; h < G; ++h) z = fmaxf(z, (sv[k][h] - mu_r[h]) * is_r[h]);
                         z = z + 0.0f;  // -0 -> +0
                         if (zrow) zrow[i] = z;
-                        if (raw_row) {
-#pragma unroll
-                            for (int h = 0; h < G; ++h) raw_row[(long long)h * a.cap_u + i] = sv[k][h];
-                        }
-                        key = float_key(z);
+                        const unsigned key = float_key(z);
                         uk[i] = key;
+                        if (selecting) atomicAdd(wh + (key >> 24), 1u);
                     }
-                    if (selecting && in) atomicAdd(wh + (key >> 24), 1u);
+                }
+            }
+            if (raw_row) {
+                for (int i = tid; i < n_local; i += kThreads) {
+                    float sv[G];
+                    load_scores<G>(sc_local + i * G, sv);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) raw_row[(long long)h * a.cap_u + i] = sv[h];
                 }
             }
         }
@@ -912,7 +925,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                     if (lane == 0) tw[wi] = __popc(bb);
                 }
                 __syncthreads();
-                const int my_ties = block_exclusive_scan(tw, nwl, iscratch);
+                const int my_ties = block_exclusive_scan<kWarps>(tw, nwl, iscratch);
                 if (tid == 0) xch->ties = my_ties;
                 cluster.sync();
                 if (tid == 0) {
@@ -948,7 +961,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
                 gpre[wg] = __popc(m);
             }
             __syncthreads();
-            const int total = block_exclusive_scan(gpre, nwt, iscratch);
+            const int total = block_exclusive_scan<kWarps>(gpre, nwt, iscratch);
             if (tid == 0) gpre[nwt] = total;
             __syncthreads();
             const int M = a.budget;
@@ -972,7 +985,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) tri_fused_kernel(const A
             // destinations, all above the destinations of round r, so the overlap is safe.
             constexpr int LPR = D / 8;  // lanes per row (16 bytes each)
             constexpr int RPW = 32 / LPR;
-            const unsigned ring_bytes = (unsigned)kWarps * nslot * kStageBytes;
+            const unsigned ring_bytes = Ly.ring_bytes;
             const int S2 = (int)((ring_bytes / 2u) / (unsigned)(4 * D + 4)) / 16 * 16;
             const unsigned buf_bytes = (unsigned)S2 * (4 * D + 4);
             const int wM = M / 32;
