@@ -28,15 +28,17 @@
 //             exchanged between the cluster's CTAs through distributed shared memory),
 //             z = (s - mu) / sigma (0 for a flat head), max over the G heads
 //             ([10100] §TriAttention方法; [Summary] §方案设计 item 4).
-//   select    top-B by max-z: four 8-bit radix passes over an order-preserving uint32
-//             image of the fp32 value, histograms merged across the cluster; exact ties
-//             at the threshold go to the lower slot.
+//   select    top-B by max-z: up to four 8-bit radix passes over an order-preserving
+//             uint32 image of the fp32 value, histograms merged across the cluster; exact
+//             ties at the threshold go to the lower slot.
 //   compact   in-place stable gather of the kept K/V/position rows to slots [0, B)
 //             ([Deep-dive] §4 prune_kv_cache: top-k then sort). Destinations are taken in
 //             rounds in ascending order; in each round every CTA first copies its
-//             sources into shared memory (cp.async), the cluster synchronises, then all
-//             CTAs write. Since a kept row never moves to a higher slot, no round can
-//             overwrite a row that this or a later round still has to read.
+//             sources into shared memory (cp.async), then writes them. A kept row never
+//             moves to a higher slot, so no round overwrites a row that a later round still
+//             has to read; only the rows that come from below slot B can be overwritten
+//             by another CTA's writes of the same round, and their rounds put a cluster
+//             barrier between the reads and the writes.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -53,7 +55,6 @@ constexpr int kBins = 256;          // radix digit width: 8 bits
 // (128 registers per thread) and 96 with 6 warps (168); GQA 8 needs the latter.
 __host__ __device__ constexpr int cta_warps(int G) { return G >= 8 ? 6 : 8; }
 __host__ __device__ constexpr int cta_threads(int G) { return cta_warps(G) * 32; }
-constexpr int kMaxWarps = 8;
 constexpr int kMinBlocks = 2;
 constexpr int kMaxCluster = 16;
 constexpr int kModePrune = 0;
@@ -233,20 +234,12 @@ __device__ __forceinline__ void st_hint(float *p, float v, uint64_t policy) {
     asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
 }
 
-__device__ __forceinline__ void st_hint_u32(unsigned *p, unsigned v, uint64_t policy) {
-    asm volatile("st.global.L2::cache_hint.b32 [%0], %1, %2;" ::"l"(p), "r"(v), "l"(policy) : "memory");
-}
-
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
 }
 
 __device__ __forceinline__ void cp_async4(void *dst_smem, const void *src) {
     asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(dst_smem)), "l"(src) : "memory");
-}
-
-__device__ __forceinline__ void cp_async_wait_all() {
-    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // Band modulus. Denormal squared norms (below 1.2e-38) flush to zero, which moves a score by
