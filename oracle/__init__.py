@@ -49,6 +49,8 @@ def _bind(L):
     L.tri_oracle_prune_batch.argtypes = [i32, i32, i32, i32, i32, i32, f64, P, i32, P,
                                          P, P, P, P, P, P, P, P, P, i32]
     L.tri_oracle_prune_batch.restype = i32
+    L.tri_oracle_calibrate.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
+    L.tri_oracle_calibrate.restype = i32
     return L
 
 
@@ -154,3 +156,21 @@ def prune_batch(K_bits, pos, lens, t, q_mean, q_norm, R, offsets, base, B, layou
     if rc != 0:
         raise ValueError("tri_oracle_prune_batch rejected its arguments")
     return kept, nk, zm
+
+
+def calibrate(Q_bits, layout=HALF, L=None):
+    """Calibration statistics from pre-RoPE query samples.
+
+    Q_bits: uint16 [L][T][Hq][d] bf16 bits. Returns fp64 (q_mean [L][Hq][d],
+    q_norm_mean [L][Hq][d/2], R [L][Hq][d/2]).
+    """
+    Lb = L or lib()
+    Q_bits = _c(Q_bits, np.uint16)
+    nl, T, Hq, d = Q_bits.shape
+    qm = np.zeros((nl, Hq, d), dtype=np.float64)
+    qn = np.zeros((nl, Hq, d // 2), dtype=np.float64)
+    R = np.zeros((nl, Hq, d // 2), dtype=np.float64)
+    rc = Lb.tri_oracle_calibrate(_p(Q_bits), nl, T, Hq, d, int(layout), _p(qm), _p(qn), _p(R))
+    if rc != 0:
+        raise ValueError("tri_oracle_calibrate: bad arguments")
+    return qm, qn, R

@@ -44,6 +44,12 @@
  * Nothing is folded, blocked or reordered beyond hoisting per-key and
  * per-head quantities out of the offset loop; the cosine series is summed
  * literally over every delta and every band.
+ *
+ * The calibration statistics the pass consumes (tri_oracle_calibrate) are the
+ * means over T calibration tokens of the pre-RoPE query bands ([Deep-dive]
+ * §3.4 offline calibration; [Stage] §TriAttention：把理论变成算法 items 1-2):
+ * the complex centre E[q_f], the mean modulus E|q_f|, and the concentration
+ * R_f = |E[q_f]| / E|q_f| of [Stage] §破局之道, taken per band.
  */
 #include <math.h>
 #include <stdint.h>
@@ -300,4 +306,46 @@ int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int lay
         free(s); free(zm);
     }
     return bad ? -1 : 0;
+}
+
+/*
+ * Calibration statistics from T pre-RoPE query samples.
+ *   Q            [L][T][Hq][d] bf16 bits of the pre-RoPE queries, in the keys' dim layout
+ *   q_mean       [L][Hq][d] out: E[q_f], its real part at band f's first dim and its
+ *                imaginary part at the second (the same layout as the queries)
+ *   q_norm_mean  [L][Hq][F] out: E|q_f|
+ *   R            [L][Hq][F] out: |E[q_f]| / E|q_f|; 0 for a band whose samples are all 0
+ *                (then E[q_f] = 0 and E|q_f| = 0 as well, so no score uses the value)
+ * Every mean is a plain average over the T tokens. Returns 0, or -1 on bad arguments.
+ */
+int tri_oracle_calibrate(const uint16_t *Q, int L, int T, int Hq, int d, int layout,
+                         double *q_mean, double *q_norm_mean, double *R)
+{
+    if (!Q || L < 1 || T < 1 || Hq < 1 || d < 2 || d % 2 || !q_mean || !q_norm_mean || !R) return -1;
+    const int F = d / 2;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int l = 0; l < L; ++l) {
+        for (int h = 0; h < Hq; ++h) {
+            for (int f = 0; f < F; ++f) {
+                int dr, di;
+                band_dims(d, layout, f, &dr, &di);
+                double sr = 0.0, si = 0.0, sm = 0.0;
+                for (int t = 0; t < T; ++t) {
+                    const uint16_t *q = Q + (((size_t)l * T + t) * Hq + h) * (size_t)d;
+                    const double re = bf16_value(q[dr]);
+                    const double im = bf16_value(q[di]);
+                    sr += re;
+                    si += im;
+                    sm += sqrt(re * re + im * im);
+                }
+                const double mr = sr / (double)T, mi = si / (double)T, mm = sm / (double)T;
+                double *qm = q_mean + ((size_t)l * Hq + h) * (size_t)d;
+                qm[dr] = mr;
+                qm[di] = mi;
+                q_norm_mean[((size_t)l * Hq + h) * F + f] = mm;
+                R[((size_t)l * Hq + h) * F + f] = mm > 0.0 ? sqrt(mr * mr + mi * mi) / mm : 0.0;
+            }
+        }
+    }
+    return 0;
 }

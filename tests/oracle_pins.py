@@ -17,6 +17,13 @@ the mathematics fix:
 * brute force on tiny inputs: the kept set is the lexicographically smallest
   of the B-subsets with the largest sum of max-z.
 
+The calibration statistics (E[q_f], E|q_f| and R_f per band from query samples) are
+pinned by a hand example (``golden/calibration_example.json``) and closed forms:
+identical tokens give R = 1, opposite tokens R = 0, two tokens of equal modulus at an
+angle theta give R = cos(theta / 2); repeating the token set changes nothing, scaling it
+by 2 scales the centre and the mean modulus and leaves R alone, and the two rotary
+layouts agree once the dims are permuted.
+
 The mutation test plants plausible mistakes in copies of the oracle and checks
 that each one trips at least one of these pins.
 """
@@ -245,6 +252,87 @@ def pin_compaction(L, seed=7):
             assert r["zmax"][kept].min() >= r["zmax"][drop].max()
 
 
+def _calib_tokens(bands, d, layout):
+    """[T][d] real vectors from [T][F][2] band samples, in the given rotary layout."""
+    bands = np.asarray(bands, dtype=np.float64)
+    T, F, _ = bands.shape
+    x = np.zeros((T, d))
+    for f, (re, im) in enumerate(_band_pairs(d, layout)):
+        x[:, re] = bands[:, f, 0]
+        x[:, im] = bands[:, f, 1]
+    return x
+
+
+def _calibrate(L, x, layout):
+    """Oracle statistics of samples x [T][d] (one layer, one head), fp64 band views."""
+    T, d = x.shape
+    qm, qn, R = oracle.calibrate(_bf16_bits(x).reshape(1, T, 1, d), layout, L=L)
+    pairs = _band_pairs(d, layout)
+    cm = np.array([[qm[0, 0, re], qm[0, 0, im]] for re, im in pairs])
+    return cm, qn[0, 0], R[0, 0]
+
+
+def pin_calibrate_hand_example(L):
+    with open(os.path.join(HERE, "golden", "calibration_example.json")) as fh:
+        g = json.load(fh)
+    for name, layout in LAYOUTS.items():
+        cm, qn, R = _calibrate(L, _calib_tokens(g["bands"], 4, layout), layout)
+        want_cm = np.array([[_expr(v) for v in b] for b in g["q_mean_bands"]])
+        assert np.allclose(cm, want_cm, rtol=0, atol=1e-15), (name, cm)
+        assert np.allclose(qn, [_expr(v) for v in g["q_norm_mean"]], rtol=0, atol=1e-14), (name, qn)
+        assert np.allclose(R, [_expr(v) for v in g["R"]], rtol=0, atol=1e-15), (name, R)
+
+
+def pin_calibrate_closed_forms(L):
+    """Identical tokens: R = 1 (0 for an all-zero band); opposite tokens: R = 0; two tokens of
+    equal modulus at angle theta: R = cos(theta / 2) (Pythagorean samples, exact in bf16)."""
+    # identical tokens, one band all zero
+    one = [[3.0, 4.0], [0.0, 0.0], [-1.5, 2.0], [5.0, -12.0]]
+    cm, qn, R = _calibrate(L, _calib_tokens([one] * 5, 8, oracle.HALF), oracle.HALF)
+    assert np.allclose(cm, one, rtol=0, atol=1e-15)
+    assert np.allclose(qn, [5.0, 0.0, 2.5, 13.0], rtol=0, atol=1e-14)
+    assert np.allclose(R, [1.0, 0.0, 1.0, 1.0], rtol=0, atol=1e-15), R
+    # opposite tokens
+    opp = [[[3.0, 4.0], [8.0, -15.0]], [[-3.0, -4.0], [-8.0, 15.0]]]
+    cm, qn, R = _calibrate(L, _calib_tokens(opp, 4, oracle.INTERLEAVED), oracle.INTERLEAVED)
+    assert np.allclose(cm, 0.0, atol=1e-15) and np.allclose(R, 0.0, atol=1e-15)
+    assert np.allclose(qn, [5.0, 17.0], rtol=0, atol=1e-14)
+    # two tokens of equal modulus: (a, b) and (b, a) for each Pythagorean pair, and (a, b), (a, -b)
+    pairs = [(3.0, 4.0), (5.0, 12.0), (8.0, 15.0), (7.0, 24.0)]
+    toks = [[[a, b] for a, b in pairs], [[b, a] for a, b in pairs]]
+    cm, qn, R = _calibrate(L, _calib_tokens(toks, 8, oracle.HALF), oracle.HALF)
+    for f, (a, b) in enumerate(pairs):
+        r = math.hypot(a, b)
+        cos_t = 2 * a * b / (r * r)
+        assert abs(R[f] - math.sqrt((1 + cos_t) / 2)) < 1e-15, (f, R[f])
+        assert abs(qn[f] - r) < 1e-13
+    toks = [[[a, b] for a, b in pairs], [[a, -b] for a, b in pairs]]
+    cm, qn, R = _calibrate(L, _calib_tokens(toks, 8, oracle.HALF), oracle.HALF)
+    for f, (a, b) in enumerate(pairs):
+        assert abs(R[f] - a / math.hypot(a, b)) < 1e-15, (f, R[f])
+
+
+def pin_calibrate_invariants(L, seed=8):
+    """Repeating the token set changes nothing; doubling every sample doubles E[q] and E|q|
+    and keeps R; the two rotary layouts give the same statistics per band."""
+    rng = np.random.default_rng(seed)
+    T, F = 37, 16
+    bands = _bf16_value(_bf16_bits(rng.normal(0.3, 1.0, (T, F, 2))))
+    for layout in LAYOUTS.values():
+        cm, qn, R = _calibrate(L, _calib_tokens(bands, 2 * F, layout), layout)
+        cm2, qn2, R2 = _calibrate(L, _calib_tokens(np.concatenate([bands, bands, bands]), 2 * F, layout), layout)
+        assert np.allclose(cm2, cm, rtol=1e-14, atol=1e-15) and np.allclose(qn2, qn, rtol=1e-14)
+        assert np.allclose(R2, R, rtol=1e-13)
+        cm3, qn3, R3 = _calibrate(L, _calib_tokens(2.0 * bands, 2 * F, layout), layout)
+        assert np.allclose(cm3, 2 * cm, rtol=1e-14, atol=1e-15) and np.allclose(qn3, 2 * qn, rtol=1e-14)
+        assert np.allclose(R3, R, rtol=1e-13)
+        assert np.all((R >= 0) & (R <= 1 + 1e-15))
+    ch, qh, Rh = _calibrate(L, _calib_tokens(bands, 2 * F, oracle.HALF), oracle.HALF)
+    ci, qi, Ri = _calibrate(L, _calib_tokens(bands, 2 * F, oracle.INTERLEAVED), oracle.INTERLEAVED)
+    assert np.array_equal(ch, ci) and np.array_equal(qh, qi) and np.array_equal(Rh, Ri)
+
+
 ALL_PINS = [pin_hand_examples, pin_rope_dot_closed_form, pin_positions_cancel,
             pin_t_shift_is_query_rotation, pin_norm_rotation_invariant_and_linear,
-            pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction]
+            pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction,
+            pin_calibrate_hand_example, pin_calibrate_closed_forms, pin_calibrate_invariants]

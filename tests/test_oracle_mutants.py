@@ -30,6 +30,14 @@ MUTANTS = {
     "qmag_not_kmag": ("series += qmag[h * F + f] * kmag[f] *", "series += qmag[h * F + f] *"),
     "flat_head_not_zero": ("const int flat = !(hi > lo);", "const int flat = 0;"),
     "no_resort": ("qsort(kept_out, (size_t)M, sizeof(int32_t), idx_cmp);", ""),
+    "calib_R_inverted": ("mm > 0.0 ? sqrt(mr * mr + mi * mi) / mm : 0.0;", "mm > 0.0 ? mm / sqrt(mr * mr + mi * mi) : 0.0;"),
+    "calib_squared_modulus": ("sm += sqrt(re * re + im * im);", "sm += re * re + im * im;"),
+    "calib_sum_not_mean": ("const double mr = sr / (double)T, mi = si / (double)T, mm = sm / (double)T;",
+                           "const double mr = sr, mi = si, mm = sm;"),
+    "calib_sample_mean_T_minus_1": ("const double mr = sr / (double)T, mi = si / (double)T, mm = sm / (double)T;",
+                                    "const double mr = sr / (double)(T - 1), mi = si / (double)(T - 1), mm = sm / (double)(T - 1);"),
+    "calib_centre_modulus_first": ("                    sr += re;\n                    si += im;",
+                                   "                    sr += fabs(re);\n                    si += fabs(im);"),
 }
 
 
