@@ -13,6 +13,12 @@ heads x GQA 4, head_dim 128, batch 4, 32768 -> 3072 keys per unit, ~19 GB of K/V
                     [--workload NAME] [--no-e2e] [--no-cpu]
 
 Prints ONE JSON line (rank 0).
+
+    python bench.py --path calibrate [--steps K] [--warmup W]
+
+measures instead the calibration-statistics estimator (tri_calibrate_estimate) on the pages'
+calibration batch (about 10K tokens through a Qwen3-8B-shaped model: 36 layers, 32 query
+heads, head_dim 128; 3 GB of bf16 pre-RoPE queries), one GPU.
 """
 from __future__ import annotations
 
@@ -441,6 +447,94 @@ def run_reference(args, rank, world):
 
 # ---------------------------------------------------------------------------------------
 
+CAL_METRIC = "calibration query rows reduced/s (Qwen3-8B shape: 36 layers x 32 heads x 128 dims per token)"
+CAL_SHAPE = (36, 10240, 32, 128)  # layers, tokens, query heads, head_dim
+
+
+def run_calibrate(args):
+    """Time tri_calibrate_estimate: CUDA events around the call (its two launches) on the
+    stream; a 256 MiB buffer is written between steps (3 GB of input exceeds L2 anyway)."""
+    import torch
+    import tri_synth as ts
+    import oracle
+    from rope_aware_key_tri_b200 import tri
+    L, T, Hq, d = CAL_SHAPE
+    if args.layers:
+        L = args.layers
+    q = ts.make_queries(L, T, Hq, d, seed=1, device="cuda")
+    ctx = tri.TriContext(0)
+    out = (torch.empty((L, Hq, d), device="cuda"), torch.empty((L, Hq, d // 2), device="cuda"),
+           torch.empty((L, Hq, d // 2), device="cuda"))
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+    for _ in range(args.warmup):
+        ctx.calibrate_estimate(q, tri.TRI_ROPE_HALF, out=out)
+    torch.cuda.synchronize()
+    times = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            ctx.calibrate_estimate(q, tri.TRI_ROPE_HALF, out=out)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    rows = L * T
+    nbytes = q.numel() * 2 + sum(x.numel() * 4 for x in out)
+    peak, kind = measured_peak()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    res = {"metric": CAL_METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp64 sums", "data": "synthetic",
+           "config": {"workload": "qwen3_8b_calibration_10k", "layers": L, "tokens": T, "q_heads": Hq,
+                      "head_dim": d, "layout": "half",
+                      "timed": "CUDA events around tri_calibrate_estimate (partial sums + means)"},
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                        "traffic": None, "algorithmic_bytes": nbytes, "peak_kind": f"{kind} (burst copy)"},
+           "clocks": clk.summary(), "gpu_launches": 2 * args.steps,
+           "ms_steps": {"min": min(times), "median": ms, "max": max(times)}}
+    if args.no_e2e:
+        ctx.close()
+        return res
+    # end to end: queries from pinned host memory, statistics back to the host
+    qh = q.cpu().pin_memory()
+    host = tuple(torch.empty(x.shape, dtype=torch.float32).pin_memory() for x in out)
+    e2e = []
+    for _ in range(2):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        q.copy_(qh, non_blocking=True)
+        ctx.calibrate_estimate(q, tri.TRI_ROPE_HALF, out=out)
+        for hx, dx in zip(host, out):
+            hx.copy_(dx, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e.append(e0.elapsed_time(e1))
+    res["e2e"] = {"value": rows / (statistics.median(e2e) * 1e-3), "unit": "rows/s",
+                  "ms_per_step": statistics.median(e2e), "h2d_bytes_per_step": q.numel() * 2,
+                  "d2h_bytes_per_step": sum(x.numel() * 4 for x in out), "steps": 2}
+    if args.no_cpu:
+        ctx.close()
+        return res
+    # the oracle on the host cores, on a bounded sample: whole layers until about 10 s
+    import numpy as np
+    dt, done = 0.0, 0
+    while done < L and dt < 10.0:
+        sub = qh[done:done + 1].contiguous().view(torch.int16).numpy().view(np.uint16)
+        t0 = time.perf_counter()
+        oracle.calibrate(sub, oracle.HALF)
+        dt += time.perf_counter() - t0
+        done += 1
+    res["cpu_baseline"] = {"value": done * T / dt, "unit": "rows/s", "cores": min(os.cpu_count() or 1, Hq),
+                           "kind": "oracle", "sample": f"{done} of {L} layers, all {Hq} heads, {T} tokens, {dt:.1f} s"}
+    ctx.close()
+    return res
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -455,8 +549,13 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--path", default="prune", choices=["prune", "calibrate"],
+                    help="prune: the scoring-and-pruning pass (default); calibrate: the statistics estimator")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.path == "calibrate":
+        print(json.dumps(run_calibrate(args)), flush=True)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

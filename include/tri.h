@@ -143,6 +143,31 @@ TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads
                               const int64_t *offsets, int n_offsets);
 
 /*
+ * Estimate the calibration statistics from pre-RoPE query samples (the pages' offline
+ * calibration step: [Deep-dive] §3.4; the statistics of [Stage] §TriAttention：把理论变成算法
+ * items 1-2 and the concentration of [Stage] §破局之道, taken per band).
+ *   Q            bf16 [n_layers][T][n_q_heads][head_dim] device: the pre-RoPE queries of T
+ *                calibration tokens, dims in the keys' rotary layout `layout`
+ *   q_mean       fp32 [n_layers][n_q_heads][head_dim] device, written: E[q_f] over the T tokens
+ *                (real part at band f's first dim, imaginary part at its second)
+ *   q_norm_mean  fp32 [n_layers][n_q_heads][head_dim/2] device, written: E|q_f|
+ *   R            fp32 [n_layers][n_q_heads][head_dim/2] device, written: |E[q_f]| / E|q_f|,
+ *                0 for a band whose samples are all zero
+ * The three outputs are what tri_calibrate_load takes (after a copy to the host).
+ * Sums run in fp64 (|q_f| from the exact bf16 components with one fp32 rounding of
+ * re^2 + im^2 and a correctly rounded fp32 square root) in a fixed order, so the results do
+ * not depend on the GPU; the outputs are rounded to fp32 once. Runs on `stream` (two launches);
+ * Q is only read. head_dim in {64, 128}; T, n_layers, n_q_heads >= 1; Q 16-byte aligned.
+ * Uses the context's scratch (grown with a device-synchronising cudaMalloc when a call needs
+ * more than any call before: n_layers * n_q_heads * head_dim/2 * ceil(T / 256) * 24 bytes).
+ * Does not need statistics to be loaded. Errors: TRI_EINVAL (argument), TRI_EUNSUPPORTED
+ * (head_dim, sizes), TRI_ENOMEM, TRI_ECUDA (tri_last_error says which call failed).
+ */
+TRI_API tri_status tri_calibrate_estimate(tri_ctx *ctx, const void *Q, int n_layers, int T, int n_q_heads,
+                                          int head_dim, tri_rope_layout layout, float *q_mean,
+                                          float *q_norm_mean, float *R, void *stream);
+
+/*
  * Score every cached key and prune each unit to its top `budget` keys, in place.
  *   t       int32 [batch] device: current query position of each sequence; the
  *           future queries are at t + delta. Positions in the cache must be < t.

@@ -19,6 +19,7 @@
 
 #include "../../include/tri.h"
 #include "tri_kernel.cuh"
+#include "tri_calib.cuh"
 
 struct tri_ctx {
     int device = -1;
@@ -552,6 +553,21 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     return TRI_OK;
 }
 
+using CalPartialFn = void (*)(const uint16_t *, int, int, int, double *);
+using CalFinalFn = void (*)(const double *, int, int, int, int, float *, float *, float *);
+
+bool pick_calib(int D, int layout, CalPartialFn *p, CalFinalFn *f) {
+#define TRI_CAL_CASE(DD, LL)                                    \
+    if (D == DD && layout == LL) {                              \
+        *p = &tri::tri_calib_partial_kernel<DD, LL>;            \
+        *f = &tri::tri_calib_final_kernel<DD, LL>;              \
+        return true;                                            \
+    }
+    TRI_CAL_CASE(64, 0) TRI_CAL_CASE(64, 1) TRI_CAL_CASE(128, 0) TRI_CAL_CASE(128, 1)
+#undef TRI_CAL_CASE
+    return false;
+}
+
 }  // namespace
 
 extern "C" {
@@ -674,6 +690,47 @@ tri_status tri_prune_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int
 
 tri_status tri_score(tri_ctx *c, const tri_kv *kv, const int32_t *t, float *raw, float *zmax, void *stream) {
     return run(c, kv, t, 0, raw, zmax, tri::kModeScore, stream);
+}
+
+tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T, int n_q_heads, int head_dim,
+                                  tri_rope_layout layout, float *q_mean, float *q_norm_mean, float *R,
+                                  void *stream) {
+    if (!c || !Q || !q_mean || !q_norm_mean || !R) return TRI_EINVAL;
+    if (n_layers < 1 || T < 1 || n_q_heads < 1) return TRI_EINVAL;
+    if (layout != TRI_ROPE_HALF && layout != TRI_ROPE_INTERLEAVED) return TRI_EINVAL;
+    CalPartialFn pk = nullptr;
+    CalFinalFn fk = nullptr;
+    if (!pick_calib(head_dim, (int)layout, &pk, &fk)) return TRI_EUNSUPPORTED;
+    if (!aligned(Q, 16) || !aligned(q_mean, 4) || !aligned(q_norm_mean, 4) || !aligned(R, 4)) return TRI_EINVAL;
+    if (!is_device_ptr(Q) || !is_device_ptr(q_mean) || !is_device_ptr(q_norm_mean) || !is_device_ptr(R))
+        return TRI_EINVAL;
+    const long long n_chunks = ((long long)T + tri::kCalChunk - 1) / tri::kCalChunk;
+    const long long bands = (long long)n_layers * n_q_heads * (head_dim / 2);
+    const long long cols = (long long)n_q_heads * (head_dim / 16);
+    const long long groups = (cols + tri::kCalThreads - 1) / tri::kCalThreads;
+    if (n_layers > 65535 || groups > 65535 || n_chunks > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+    const size_t need = (size_t)n_chunks * (size_t)bands * 3 * sizeof(double);
+    if (need > c->scratch_bytes) {
+        cudaFree(c->d_scratch);  // synchronises the device: no call still uses the old scratch
+        c->d_scratch = nullptr;
+        c->scratch_bytes = 0;
+        ce = cudaMalloc(&c->d_scratch, need);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaMalloc(scratch)", TRI_ENOMEM);
+        c->scratch_bytes = need;
+    }
+    double *part = reinterpret_cast<double *>(c->d_scratch);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const dim3 grid1((unsigned)n_chunks, (unsigned)n_layers, (unsigned)groups);
+    pk<<<grid1, tri::kCalThreads, 0, st>>>(static_cast<const uint16_t *>(Q), n_layers, T, n_q_heads, part);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "calibration partial sums");
+    const dim3 grid2((unsigned)((bands + tri::kCalThreads - 1) / tri::kCalThreads));
+    fk<<<grid2, tri::kCalThreads, 0, st>>>(part, (int)n_chunks, n_layers, T, n_q_heads, q_mean, q_norm_mean, R);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "calibration means");
+    return TRI_OK;
 }
 
 tri_status tri_set_tuning(tri_ctx *c, int cluster_size, int buffers_per_warp) {

@@ -1,0 +1,140 @@
+// tri_calib.cuh -- calibration statistics from pre-RoPE query samples, for sm_100a.
+//
+// Pages cited (titles; sections as headed on each page):
+//   [Deep-dive]  "TriAttention深度解析：用三角函数革命性压缩KV Cache，让长推理从「显存地狱」中脱困"
+//   [Stage]      "旋转舞台上的追光者——TriAttention如何用三角函数破解长文本推理的内存困局"
+//
+// The offline calibration of [Deep-dive] §3.4 runs a small batch (about 10K tokens) through
+// the model and keeps, per attention head, the query centre, the mean norm and the
+// concentration R. Per band f of query head h of layer l, over the T calibration tokens:
+//   E[q_f]  = mean_t q_f(t)                  (complex; [Stage] §TriAttention：把理论变成算法 item 1)
+//   E|q_f|  = mean_t |q_f(t)|                ([Stage] item 2)
+//   R_f     = |E[q_f]| / E|q_f|              ([Stage] §破局之道, taken per band; 0 for a band
+//                                            whose samples are all zero)
+//
+// The pass is one stream over Q (HBM-bound): a CTA takes a fixed chunk of tokens of one
+// layer and one group of 128 sixteen-byte columns; each thread owns 8 bands of one head
+// (two 16-byte pieces per token: the band's two dims sit 64 dims apart in the half layout,
+// side by side in the interleaved one), sums re, im in fp64 and |q_f| (from the exact bf16
+// components: one fp32 rounding of re^2 + im^2, a correctly rounded fp32 square root) in
+// fp64, and writes its chunk's sums; 8 tokens are loaded before any is used, so a thread
+// keeps 256 bytes in flight. A second launch adds the chunks in order, so the result does
+// not depend on the GPU, and forms the means and R.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace tri {
+
+constexpr int kCalThreads = 128;
+constexpr int kCalChunk = 256;  // tokens per partial sum (fixed: the summation order is part of the result)
+constexpr int kCalUnroll = 8;   // tokens in flight per thread (16 loads of 16 bytes)
+
+__device__ __forceinline__ float cal_lo(unsigned w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float cal_hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
+
+// part: [n_chunks][L][Hq][F][3] fp64 (sum re, sum im, sum |q_f|)
+template <int D, int LAYOUT>
+__global__ void __launch_bounds__(kCalThreads, 3) tri_calib_partial_kernel(const uint16_t *__restrict__ Q, int L,
+                                                                        int T, int Hq,
+                                                                        double *__restrict__ part) {
+    constexpr int F = D / 2;
+    constexpr int SLOTS = D / 16;  // 16-dim column slots per head: 8 bands each
+    const int col = blockIdx.z * kCalThreads + threadIdx.x;
+    if (col >= Hq * SLOTS) return;  // no barrier in this kernel
+    const int chunk = blockIdx.x, l = blockIdx.y;
+    const int h = col / SLOTS, slot = col % SLOTS;
+    const int t0 = chunk * kCalChunk;
+    const int t1 = min(T, t0 + kCalChunk);
+    // element offsets of the thread's two 16-byte pieces in a token row
+    const int off_a = LAYOUT == 0 ? h * D + slot * 8 : h * D + slot * 16;
+    const int off_b = LAYOUT == 0 ? off_a + F : off_a + 8;
+    const size_t row = (size_t)Hq * D;
+    const uint16_t *base = Q + (size_t)l * T * row;
+
+    double sr[8], si[8], sm[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) sr[k] = si[k] = sm[k] = 0.0;
+    // one token's two pieces into the band sums
+    auto add = [&](uint4 va, uint4 vb) {
+        const unsigned wa[4] = {va.x, va.y, va.z, va.w};
+        const unsigned wb[4] = {vb.x, vb.y, vb.z, vb.w};
+        float re[8], im[8];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            if (LAYOUT == 0) {
+                // piece a: re of bands 2k, 2k+1; piece b: their im
+                re[2 * k] = cal_lo(wa[k]);
+                re[2 * k + 1] = cal_hi(wa[k]);
+                im[2 * k] = cal_lo(wb[k]);
+                im[2 * k + 1] = cal_hi(wb[k]);
+            } else {
+                // each word is one band (re, im); piece a: bands 0..3, piece b: 4..7
+                re[k] = cal_lo(wa[k]);
+                im[k] = cal_hi(wa[k]);
+                re[4 + k] = cal_lo(wb[k]);
+                im[4 + k] = cal_hi(wb[k]);
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            sr[k] += (double)re[k];
+            si[k] += (double)im[k];
+            sm[k] += (double)__fsqrt_rn(fmaf(re[k], re[k], im[k] * im[k]));
+        }
+    };
+    int t = t0;
+    // whole batches: every load of the batch in flight before the first is used
+    for (; t + kCalUnroll <= t1; t += kCalUnroll) {
+        uint4 va[kCalUnroll], vb[kCalUnroll];
+#pragma unroll
+        for (int u = 0; u < kCalUnroll; ++u) {
+            const uint16_t *r = base + (size_t)(t + u) * row;
+            va[u] = __ldg(reinterpret_cast<const uint4 *>(r + off_a));
+            vb[u] = __ldg(reinterpret_cast<const uint4 *>(r + off_b));
+        }
+#pragma unroll
+        for (int u = 0; u < kCalUnroll; ++u) add(va[u], vb[u]);
+    }
+    for (; t < t1; ++t) {  // the chunk's ragged tail (the last chunk of a layer only)
+        const uint16_t *r = base + (size_t)t * row;
+        add(__ldg(reinterpret_cast<const uint4 *>(r + off_a)), __ldg(reinterpret_cast<const uint4 *>(r + off_b)));
+    }
+    double *p = part + ((((size_t)chunk * L + l) * Hq + h) * F + (size_t)slot * 8) * 3;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        p[3 * k] = sr[k];
+        p[3 * k + 1] = si[k];
+        p[3 * k + 2] = sm[k];
+    }
+}
+
+// One thread per (layer, head, band): chunk sums added in chunk order, then the means.
+template <int D, int LAYOUT>
+__global__ void __launch_bounds__(kCalThreads) tri_calib_final_kernel(const double *__restrict__ part, int n_chunks,
+                                                                      int L, int T, int Hq, float *q_mean,
+                                                                      float *q_norm_mean, float *R) {
+    constexpr int F = D / 2;
+    const long long i = (long long)blockIdx.x * kCalThreads + threadIdx.x;
+    const long long nb = (long long)L * Hq * F;
+    if (i >= nb) return;
+    const int f = (int)(i % F);
+    const long long lh = i / F;  // l * Hq + h
+    double sr = 0.0, si = 0.0, sm = 0.0;
+    for (int c = 0; c < n_chunks; ++c) {
+        const double *p = part + ((size_t)c * nb + (size_t)i) * 3;
+        sr += p[0];
+        si += p[1];
+        sm += p[2];
+    }
+    const double mr = sr / (double)T, mi = si / (double)T, mm = sm / (double)T;
+    const int dre = LAYOUT == 0 ? f : 2 * f;
+    const int dim = LAYOUT == 0 ? f + F : 2 * f + 1;
+    q_mean[lh * D + dre] = (float)mr;
+    q_mean[lh * D + dim] = (float)mi;
+    q_norm_mean[i] = (float)mm;
+    R[i] = mm > 0.0 ? (float)(sqrt(mr * mr + mi * mi) / mm) : 0.0f;
+}
+
+}  // namespace tri

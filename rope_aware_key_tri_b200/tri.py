@@ -62,6 +62,8 @@ def _load():
     L.tri_prune.argtypes = [P, ctypes.POINTER(tri_kv), P, I32, P]
     L.tri_prune_noalloc.argtypes = [P, ctypes.POINTER(tri_kv), P, I32, P]
     L.tri_score.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
+    L.tri_calibrate_estimate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                         ctypes.c_int, P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
     L.tri_set_tuning.argtypes = [P, ctypes.c_int, ctypes.c_int]
     L.tri_last_error.argtypes = [P]
@@ -69,7 +71,7 @@ def _load():
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
     for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
-               "tri_get_error", "tri_set_tuning", "tri_version"):
+               "tri_calibrate_estimate", "tri_get_error", "tri_set_tuning", "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
     return L
 
@@ -128,6 +130,12 @@ def tri_prune_noalloc(ctx, kv: tri_kv, t_ptr: int, budget: int, stream: int) -> 
 
 def tri_score(ctx, kv: tri_kv, t_ptr: int, raw_ptr: int, zmax_ptr: int, stream: int) -> int:
     return _lib.tri_score(ctx, ctypes.byref(kv), t_ptr, raw_ptr, zmax_ptr, stream)
+
+
+def tri_calibrate_estimate(ctx, q_ptr: int, n_layers: int, T: int, n_q_heads: int, head_dim: int, layout: int,
+                           q_mean_ptr: int, q_norm_mean_ptr: int, R_ptr: int, stream: int) -> int:
+    return _lib.tri_calibrate_estimate(ctx, q_ptr, int(n_layers), int(T), int(n_q_heads), int(head_dim),
+                                       int(layout), q_mean_ptr, q_norm_mean_ptr, R_ptr, stream)
 
 
 def tri_get_error(ctx, stream: int):
@@ -247,6 +255,26 @@ class TriContext:
         if check and st != TRI_OK:
             raise TriError(st, "tri_score", tri_last_error(self.handle))
         return st
+
+    def calibrate_estimate(self, Q, layout, out=None, stream=None, check=True):
+        """Calibration statistics from pre-RoPE queries Q (bf16 [n_layers][T][n_q_heads][head_dim],
+        on this context's device). Returns fp32 device tensors (q_mean [L][Hq][d],
+        q_norm_mean [L][Hq][d/2], R [L][Hq][d/2]), or the status when check is False."""
+        if Q.dtype != torch.bfloat16 or Q.dim() != 4 or not Q.is_contiguous():
+            raise TriError(TRI_EINVAL, "tri_calibrate_estimate", "Q must be a contiguous bf16 [L][T][Hq][d] tensor")
+        nl, T, Hq, d = Q.shape
+        if out is None:
+            out = (torch.empty((nl, Hq, d), dtype=torch.float32, device=Q.device),
+                   torch.empty((nl, Hq, d // 2), dtype=torch.float32, device=Q.device),
+                   torch.empty((nl, Hq, d // 2), dtype=torch.float32, device=Q.device))
+        qm, qn, R = out
+        st = tri_calibrate_estimate(self.handle, Q.data_ptr(), nl, T, Hq, d, int(layout), qm.data_ptr(),
+                                    qn.data_ptr(), R.data_ptr(), _stream_handle(stream))
+        if not check:
+            return st
+        if st != TRI_OK:
+            raise TriError(st, "tri_calibrate_estimate", tri_last_error(self.handle))
+        return qm, qn, R
 
     def get_error(self, stream=None):
         return tri_get_error(self.handle, _stream_handle(stream))

@@ -352,3 +352,27 @@ def make_cache(spec: CacheSpec, seed: int, device="cpu", lens=None, t=None,
 
 def replace(spec: CacheSpec, **kw) -> CacheSpec:
     return dataclasses.replace(spec, **kw)
+
+
+def make_queries(n_layers: int, T: int, n_q_heads: int, head_dim: int, seed: int,
+                 sigma=(0.05, 1.5), device="cpu") -> torch.Tensor:
+    """Pre-RoPE query samples for calibration: bf16 [n_layers][T][n_q_heads][head_dim].
+
+    Per (layer, head) a centre drawn N(0, 1) per dim and a spread drawn U[sigma]; every token
+    is centre + spread * N(0, 1) per dim, so heads range from tightly concentrated to diffuse.
+    One band of head 0 in every layer is all zero (the degenerate band).
+    """
+    gen = torch.Generator().manual_seed(seed * 104729 + 3)
+    c = torch.randn((n_layers, 1, n_q_heads, head_dim), generator=gen)
+    sp = sigma[0] + (sigma[1] - sigma[0]) * torch.rand((n_layers, 1, n_q_heads, 1), generator=gen)
+    q = torch.empty((n_layers, T, n_q_heads, head_dim), dtype=torch.bfloat16)
+    step = max(1, (1 << 24) // max(1, n_q_heads * head_dim))
+    for l in range(n_layers):
+        for t0 in range(0, T, step):
+            t1 = min(T, t0 + step)
+            z = torch.randn((t1 - t0, n_q_heads, head_dim), generator=gen)
+            q[l, t0:t1] = (c[l] + sp[l] * z).to(torch.bfloat16)
+    q[:, :, 0, 0] = 0
+    q[:, :, 0, head_dim // 2] = 0
+    q[:, :, 0, 1] = 0
+    return q.to(device)
