@@ -706,7 +706,7 @@ tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T
         return TRI_EINVAL;
     const long long n_chunks = ((long long)T + tri::kCalChunk - 1) / tri::kCalChunk;
     const long long bands = (long long)n_layers * n_q_heads * (head_dim / 2);
-    const long long cols = (long long)n_q_heads * (head_dim / 16);
+    const long long cols = (long long)n_q_heads * (head_dim / 2 / tri::kCalBands);
     const long long groups = (cols + tri::kCalThreads - 1) / tri::kCalThreads;
     if (n_layers > 65535 || groups > 65535 || n_chunks > 0x7fffffffLL) return TRI_EUNSUPPORTED;
     cudaError_t ce = cudaSetDevice(c->device);

@@ -13,13 +13,12 @@
 //                                            whose samples are all zero)
 //
 // The pass is one stream over Q (HBM-bound): a CTA takes a fixed chunk of tokens of one
-// layer and one group of 128 sixteen-byte columns; each thread owns 8 bands of one head
-// (two 16-byte pieces per token: the band's two dims sit 64 dims apart in the half layout,
-// side by side in the interleaved one), sums re, im in fp64 and |q_f| (from the exact bf16
-// components: one fp32 rounding of re^2 + im^2, a correctly rounded fp32 square root) in
-// fp64, and writes its chunk's sums; 8 tokens are loaded before any is used, so a thread
-// keeps 256 bytes in flight. A second launch adds the chunks in order, so the result does
-// not depend on the GPU, and forms the means and R.
+// layer and 128 threads; each thread owns 4 bands of one head (16 bytes per token: two 8-byte
+// pieces in the half layout, where a band's two dims sit d/2 apart, one 16-byte piece in the
+// interleaved layout), sums re, im in fp64 and |q_f| (from the exact bf16 components: one
+// fp32 rounding of re^2 + im^2, a correctly rounded fp32 square root) in fp64, and writes its
+// chunk's sums; 8 tokens are loaded before any is used. A second launch adds the chunks in
+// order, so the result does not depend on the GPU, and forms the means and R.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -28,82 +27,87 @@
 namespace tri {
 
 constexpr int kCalThreads = 128;
-constexpr int kCalChunk = 256;  // tokens per partial sum (fixed: the summation order is part of the result)
-constexpr int kCalUnroll = 8;   // tokens in flight per thread (16 loads of 16 bytes)
+constexpr int kCalMinBlocks = 6;  // CTAs per SM (24 warps hide the fp64 dependency latency)
+constexpr int kCalBands = 4;      // bands per thread
+constexpr int kCalChunk = 256;    // tokens per partial sum (fixed: the summation order is part of the result)
+constexpr int kCalUnroll = 8;     // tokens in flight per thread
 
 __device__ __forceinline__ float cal_lo(unsigned w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float cal_hi(unsigned w) { return __uint_as_float(w & 0xffff0000u); }
 
 // part: [n_chunks][L][Hq][F][3] fp64 (sum re, sum im, sum |q_f|)
+// A thread owns kCalBands bands of one head: its re and im dims are two 8-byte pieces in the
+// half layout (d/2 dims apart) and one 16-byte piece in the interleaved layout.
 template <int D, int LAYOUT>
-__global__ void __launch_bounds__(kCalThreads, 3) tri_calib_partial_kernel(const uint16_t *__restrict__ Q, int L,
-                                                                        int T, int Hq,
-                                                                        double *__restrict__ part) {
+__global__ void __launch_bounds__(kCalThreads, kCalMinBlocks) tri_calib_partial_kernel(const uint16_t *__restrict__ Q,
+                                                                                    int L, int T, int Hq,
+                                                                                    double *__restrict__ part) {
     constexpr int F = D / 2;
-    constexpr int SLOTS = D / 16;  // 16-dim column slots per head: 8 bands each
+    constexpr int NB = kCalBands;
+    constexpr int SLOTS = F / NB;  // column slots per head
     const int col = blockIdx.z * kCalThreads + threadIdx.x;
     if (col >= Hq * SLOTS) return;  // no barrier in this kernel
     const int chunk = blockIdx.x, l = blockIdx.y;
     const int h = col / SLOTS, slot = col % SLOTS;
     const int t0 = chunk * kCalChunk;
     const int t1 = min(T, t0 + kCalChunk);
-    // element offsets of the thread's two 16-byte pieces in a token row
-    const int off_a = LAYOUT == 0 ? h * D + slot * 8 : h * D + slot * 16;
-    const int off_b = LAYOUT == 0 ? off_a + F : off_a + 8;
+    // element offset of the thread's re piece (half) or band piece (interleaved) in a token row
+    const int off = LAYOUT == 0 ? h * D + slot * NB : h * D + slot * 2 * NB;
     const size_t row = (size_t)Hq * D;
     const uint16_t *base = Q + (size_t)l * T * row;
 
-    double sr[8], si[8], sm[8];
+    double sr[NB], si[NB], sm[NB];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) sr[k] = si[k] = sm[k] = 0.0;
-    // one token's two pieces into the band sums
-    auto add = [&](uint4 va, uint4 vb) {
-        const unsigned wa[4] = {va.x, va.y, va.z, va.w};
-        const unsigned wb[4] = {vb.x, vb.y, vb.z, vb.w};
-        float re[8], im[8];
+    for (int k = 0; k < NB; ++k) sr[k] = si[k] = sm[k] = 0.0;
+    // one token's pieces (four 32-bit words: 4 bands) into the band sums
+    auto add = [&](uint4 w) {
+        const unsigned wv[4] = {w.x, w.y, w.z, w.w};
+        float re[NB], im[NB];
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < 2; ++k) {
             if (LAYOUT == 0) {
-                // piece a: re of bands 2k, 2k+1; piece b: their im
-                re[2 * k] = cal_lo(wa[k]);
-                re[2 * k + 1] = cal_hi(wa[k]);
-                im[2 * k] = cal_lo(wb[k]);
-                im[2 * k + 1] = cal_hi(wb[k]);
+                // words 0-1: re of bands 0..3; words 2-3: their im
+                re[2 * k] = cal_lo(wv[k]);
+                re[2 * k + 1] = cal_hi(wv[k]);
+                im[2 * k] = cal_lo(wv[2 + k]);
+                im[2 * k + 1] = cal_hi(wv[2 + k]);
             } else {
-                // each word is one band (re, im); piece a: bands 0..3, piece b: 4..7
-                re[k] = cal_lo(wa[k]);
-                im[k] = cal_hi(wa[k]);
-                re[4 + k] = cal_lo(wb[k]);
-                im[4 + k] = cal_hi(wb[k]);
+                // each word is one band (re, im)
+                re[2 * k] = cal_lo(wv[2 * k]);
+                im[2 * k] = cal_hi(wv[2 * k]);
+                re[2 * k + 1] = cal_lo(wv[2 * k + 1]);
+                im[2 * k + 1] = cal_hi(wv[2 * k + 1]);
             }
         }
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int k = 0; k < NB; ++k) {
             sr[k] += (double)re[k];
             si[k] += (double)im[k];
             sm[k] += (double)__fsqrt_rn(fmaf(re[k], re[k], im[k] * im[k]));
         }
     };
+    auto load = [&](int t) {
+        const uint16_t *r = base + (size_t)t * row + off;
+        if (LAYOUT == 0) {
+            const uint2 a = __ldg(reinterpret_cast<const uint2 *>(r));
+            const uint2 b = __ldg(reinterpret_cast<const uint2 *>(r + F));
+            return make_uint4(a.x, a.y, b.x, b.y);
+        }
+        return __ldg(reinterpret_cast<const uint4 *>(r));
+    };
     int t = t0;
     // whole batches: every load of the batch in flight before the first is used
     for (; t + kCalUnroll <= t1; t += kCalUnroll) {
-        uint4 va[kCalUnroll], vb[kCalUnroll];
+        uint4 v[kCalUnroll];
 #pragma unroll
-        for (int u = 0; u < kCalUnroll; ++u) {
-            const uint16_t *r = base + (size_t)(t + u) * row;
-            va[u] = __ldg(reinterpret_cast<const uint4 *>(r + off_a));
-            vb[u] = __ldg(reinterpret_cast<const uint4 *>(r + off_b));
-        }
+        for (int u = 0; u < kCalUnroll; ++u) v[u] = load(t + u);
 #pragma unroll
-        for (int u = 0; u < kCalUnroll; ++u) add(va[u], vb[u]);
+        for (int u = 0; u < kCalUnroll; ++u) add(v[u]);
     }
-    for (; t < t1; ++t) {  // the chunk's ragged tail (the last chunk of a layer only)
-        const uint16_t *r = base + (size_t)t * row;
-        add(__ldg(reinterpret_cast<const uint4 *>(r + off_a)), __ldg(reinterpret_cast<const uint4 *>(r + off_b)));
-    }
-    double *p = part + ((((size_t)chunk * L + l) * Hq + h) * F + (size_t)slot * 8) * 3;
+    for (; t < t1; ++t) add(load(t));  // the chunk's ragged tail (the last chunk of a layer only)
+    double *p = part + ((((size_t)chunk * L + l) * Hq + h) * F + (size_t)slot * NB) * 3;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < NB; ++k) {
         p[3 * k] = sr[k];
         p[3 * k + 1] = si[k];
         p[3 * k + 2] = sm[k];
