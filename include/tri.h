@@ -37,8 +37,9 @@
  *     sequence is left untouched. Kernels never trap.
  *   - A context is bound to one device and is not thread-safe: serialise calls
  *     that share a context. Calls that share a context but run on different
- *     streams must not overlap on the GPU (they share the status word and the
- *     completion counter).
+ *     streams must not overlap on the GPU (they share the status word, the
+ *     completion counter and the scratch that tri_prune, tri_score and
+ *     tri_calibrate_estimate use).
  */
 #ifndef TRI_H_
 #define TRI_H_
