@@ -19,6 +19,13 @@ Prints ONE JSON line (rank 0).
 measures instead the calibration-statistics estimator (tri_calibrate_estimate) on the pages'
 calibration batch (about 10K tokens through a Qwen3-8B-shaped model: 36 layers, 32 query
 heads, head_dim 128; 3 GB of bf16 pre-RoPE queries), one GPU.
+
+    python bench.py --path decode [--steps K] [--warmup W]
+
+measures the decode loop's cache maintenance in steady state on the periodic Qwen3-8B workload
+(36 layers x 8 KV heads, batch 8, budget 3072, paged with 64-token pages): one cycle = 128
+tri_append calls (one token for every sequence each) and one tri_prune (3200 -> 3072 keys per
+unit), with the pages freed by the prune returned to a free list and handed out again.
 """
 from __future__ import annotations
 
@@ -535,6 +542,106 @@ def run_calibrate(args):
     return res
 
 
+DEC_METRIC = "decode-loop cache maintenance: generated tokens/s (128 appends + 1 prune per 128 tokens, Qwen3-8B shape)"
+
+
+def run_decode(args):
+    """One timed step = one cadence cycle (128 appends, then the prune), CUDA events around the
+    cycle on the stream; the block-table updates of the cycle (host writes, one copy to the
+    device per page boundary) are inside it. The cache carries over from cycle to cycle: the
+    prune brings every sequence back to B, the next 128 appends grow it to B + 128."""
+    import numpy as np
+    import torch
+    import tri_synth as ts
+    from rope_aware_key_tri_b200 import tri
+    spec = ts.WORKLOADS["qwen3_8b_periodic_36l_3200"]
+    L, Hkv, G, d, batch, B, cad = spec.n_layers, spec.n_kv_heads, spec.group, spec.head_dim, spec.batch, \
+        spec.budget, 128
+    if args.layers:
+        L = args.layers
+    ps = 64
+    max_pages = (B + cad + ps - 1) // ps
+    n_pages = batch * max_pages + batch
+    g = torch.Generator(device="cuda").manual_seed(7)
+    K = (torch.randn((L, n_pages, Hkv, ps, d), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    V = torch.randn((L, n_pages, Hkv, ps, d), generator=g, device="cuda").to(torch.bfloat16)
+    P = torch.zeros((L, n_pages, Hkv, ps), dtype=torch.int32, device="cuda")
+    # sequence s starts at B tokens (positions 0..B-1) in pages s*max_pages + j
+    bt = np.full((batch, max_pages), -1, dtype=np.int32)
+    free = list(range(n_pages))
+    for s in range(batch):
+        for j in range((B + ps - 1) // ps):
+            bt[s, j] = free.pop(0)
+    slot = torch.arange(ps, device="cuda", dtype=torch.int32)
+    for s in range(batch):
+        for j in range((B + ps - 1) // ps):
+            P[:, int(bt[s, j]), :, :] = (j * ps + slot)[None, None, :]
+    bt_dev = torch.from_numpy(bt).cuda()
+    lens = torch.full((batch,), B, dtype=torch.int32, device="cuda")
+    tpos = torch.full((batch,), B, dtype=torch.int32, device="cuda")
+    qm, qn, R, offsets = ts.make_stats(ts.replace(spec, n_layers=L), 1)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(L, Hkv, G, d, spec.rope_base, spec.layout, qm, qn, R, offsets)
+    new_k = (torch.randn((cad, L, batch, Hkv, d), generator=g, device="cuda") * 0.5).to(torch.bfloat16)
+    new_v = torch.randn((cad, L, batch, Hkv, d), generator=g, device="cuda").to(torch.bfloat16)
+    host_len = B
+    stream = torch.cuda.current_stream()
+
+    def cycle():
+        nonlocal host_len
+        for i in range(cad):
+            if host_len % ps == 0:  # every sequence needs its next page
+                for s in range(batch):
+                    bt[s, host_len // ps] = free.pop(0)
+                bt_dev.copy_(torch.from_numpy(bt))  # from pageable memory: the host waits for it
+            ctx.append(K, V, P, lens, bt_dev, new_k[i], new_v[i], tpos)
+            tpos.add_(1)
+            host_len += 1
+        ctx.prune(K, V, P, lens, tpos, B, block_table=bt_dev)
+        host_len = B
+        for s in range(batch):  # pages past B go back to the free list
+            for j in range((B + ps - 1) // ps, max_pages):
+                if bt[s, j] >= 0:
+                    free.append(int(bt[s, j]))
+                    bt[s, j] = -1
+        bt_dev.copy_(torch.from_numpy(bt))
+
+    for _ in range(args.warmup):
+        cycle()
+    torch.cuda.synchronize()
+    assert ctx.get_error()[0] == tri.TRI_OK
+    times = []
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        for _ in range(args.steps):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            cycle()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+    st = ctx.get_error()
+    assert st[0] == tri.TRI_OK, st
+    assert torch.all(lens == B)
+    ms = statistics.median(times)
+    row = d * 2
+    units = L * batch * Hkv
+    nbytes = cad * units * (2 * row + 4) + algorithmic_bytes([B + cad] * batch, L, Hkv, d, B)
+    peak, kind = measured_peak()
+    achieved = nbytes / (ms * 1e-3) / 1e9
+    ctx.close()
+    return {"metric": DEC_METRIC, "value": batch * cad / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "qwen3_8b_periodic_36l_3200 (paged, 64-token pages)", "layers": L,
+                       "kv_heads": Hkv, "group": G, "head_dim": d, "batch": batch, "budget": B, "cadence": cad,
+                       "timed": "CUDA events around one cycle: 128 tri_append + block-table copies + tri_prune"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": None, "algorithmic_bytes": nbytes, "peak_kind": f"{kind} (burst copy)"},
+            "clocks": clk.summary(), "gpu_launches": (2 * cad + 1) * args.steps,
+            "ms_steps": {"min": min(times), "median": ms, "max": max(times)}}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -549,12 +656,16 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--path", default="prune", choices=["prune", "calibrate"],
-                    help="prune: the scoring-and-pruning pass (default); calibrate: the statistics estimator")
+    ap.add_argument("--path", default="prune", choices=["prune", "calibrate", "decode"],
+                    help="prune: the scoring-and-pruning pass (default); calibrate: the statistics estimator; "
+                         "decode: the decode loop's appends and prunes")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.path == "calibrate":
         print(json.dumps(run_calibrate(args)), flush=True)
+        return
+    if args.path == "decode":
+        print(json.dumps(run_decode(args)), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))

@@ -144,6 +144,27 @@ TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads
                               const int64_t *offsets, int n_offsets);
 
 /*
+ * Append one token to every sequence of a paged cache: the decode loop's write between two
+ * prunes, which the caller runs once every 128 generated tokens ([10100] §TriAttention方法;
+ * [Summary] §方案设计 item 4).
+ *   kv       paged cache (block_table required); its n_layers layers, lens and lens_out
+ *   K_new, V_new  bf16 [n_layers][batch][n_kv_heads][head_dim] device, 16-byte aligned: the
+ *            new token's key and value rows (the key after RoPE, like the cached ones)
+ *   pos_new  int32 [batch] device: the new token's position in each sequence
+ * Slot lens[s] of every unit of sequence s receives the rows and the position, and
+ * lens_out[s] = lens[s] + 1 (lens_out may alias lens; it is required here). The page that
+ * slot lands in, block_table[s][lens[s] / page_size], must already be allocated by the
+ * caller (an id in [0, n_pages)); freeing the pages past a sequence's length after a prune
+ * is the caller's business too. A sequence whose slot is past its capacity or lands in an
+ * unallocated page is refused as a whole (lens_out[s] = lens[s]; tri_get_error reports
+ * TRI_DEV_LEN_GT_CAP or TRI_DEV_BAD_PAGE); a refused sequence may have received the rows of
+ * some layers before the refusal. Needs the statistics loaded (for n_kv_heads and head_dim).
+ * Two launches on `stream`.
+ */
+TRI_API tri_status tri_append(tri_ctx *ctx, const tri_kv *kv, const void *K_new, const void *V_new,
+                              const int32_t *pos_new, void *stream);
+
+/*
  * Estimate the calibration statistics from pre-RoPE query samples (the pages' offline
  * calibration step: [Deep-dive] §3.4; the statistics of [Stage] §TriAttention：把理论变成算法
  * items 1-2 and the concentration of [Stage] §破局之道, taken per band).

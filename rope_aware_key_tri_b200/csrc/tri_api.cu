@@ -20,6 +20,7 @@
 #include "../../include/tri.h"
 #include "tri_kernel.cuh"
 #include "tri_calib.cuh"
+#include "tri_append.cuh"
 
 struct tri_ctx {
     int device = -1;
@@ -730,6 +731,66 @@ tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T
     fk<<<grid2, tri::kCalThreads, 0, st>>>(part, (int)n_chunks, n_layers, T, n_q_heads, q_mean, q_norm_mean, R);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "calibration means");
+    return TRI_OK;
+}
+
+tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, const int32_t *pos_new,
+                      void *stream) {
+    if (!c || !kv || !K_new || !V_new || !pos_new) return TRI_EINVAL;
+    if (!c->loaded) return TRI_ESTATE;
+    if (c->D != 64 && c->D != 128) return TRI_EUNSUPPORTED;
+    if (!kv->block_table || !kv->K || !kv->V || !kv->pos || !kv->lens || !kv->lens_out) return TRI_EINVAL;
+    if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
+        return TRI_EINVAL;
+    if (kv->page_size < 16 || kv->page_size % 16 != 0 || kv->max_pages < 1 || kv->n_pages < 1) return TRI_EINVAL;
+    const void *dev[] = {kv->K, kv->V, kv->pos, kv->lens, kv->lens_out, kv->block_table, K_new, V_new, pos_new};
+    for (const void *p : dev)
+        if (!is_device_ptr(p)) return TRI_EINVAL;
+    if (!aligned(kv->K, 16) || !aligned(kv->V, 16) || !aligned(K_new, 16) || !aligned(V_new, 16) ||
+        !aligned(kv->pos, 4) || !aligned(kv->lens, 4) || !aligned(kv->lens_out, 4) || !aligned(pos_new, 4) ||
+        !aligned(kv->block_table, 4))
+        return TRI_EINVAL;
+    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
+    if ((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+    if (kv->batch > c->seq_bad_cap) {
+        cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
+        c->d_seq_bad = nullptr;
+        c->seq_bad_cap = 0;
+        if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ENOMEM;
+        if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ECUDA;
+        c->seq_bad_cap = kv->batch;
+    }
+    tri::AppendArgs a;
+    a.K = static_cast<uint16_t *>(kv->K);
+    a.V = static_cast<uint16_t *>(kv->V);
+    a.pos = kv->pos;
+    a.K_new = static_cast<const uint16_t *>(K_new);
+    a.V_new = static_cast<const uint16_t *>(V_new);
+    a.pos_new = pos_new;
+    a.lens = kv->lens;
+    a.block_table = kv->block_table;
+    a.batch = kv->batch;
+    a.n_kv = c->Hkv;
+    a.n_layers = kv->n_layers;
+    a.page_size = kv->page_size;
+    a.max_pages = kv->max_pages;
+    a.n_pages = kv->n_pages;
+    a.status = c->d_status;
+    a.seq_bad = c->d_seq_bad;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
+    if (c->D == 128)
+        tri::tri_append_kernel<128><<<blocks, tri::kAppendWarps * 32, 0, st>>>(a);
+    else
+        tri::tri_append_kernel<64><<<blocks, tri::kAppendWarps * 32, 0, st>>>(a);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "append rows");
+    tri::tri_append_lens_kernel<<<(unsigned)((kv->batch + 255) / 256), 256, 0, st>>>(kv->lens, kv->lens_out,
+                                                                                       c->d_seq_bad, kv->batch);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "append lengths");
     return TRI_OK;
 }
 

@@ -64,6 +64,7 @@ def _load():
     L.tri_score.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_calibrate_estimate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, P, P, P, P]
+    L.tri_append.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
     L.tri_set_tuning.argtypes = [P, ctypes.c_int, ctypes.c_int]
     L.tri_last_error.argtypes = [P]
@@ -71,7 +72,7 @@ def _load():
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
     for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
-               "tri_calibrate_estimate", "tri_get_error", "tri_set_tuning", "tri_version"):
+               "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_set_tuning", "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
     return L
 
@@ -136,6 +137,10 @@ def tri_calibrate_estimate(ctx, q_ptr: int, n_layers: int, T: int, n_q_heads: in
                            q_mean_ptr: int, q_norm_mean_ptr: int, R_ptr: int, stream: int) -> int:
     return _lib.tri_calibrate_estimate(ctx, q_ptr, int(n_layers), int(T), int(n_q_heads), int(head_dim),
                                        int(layout), q_mean_ptr, q_norm_mean_ptr, R_ptr, stream)
+
+
+def tri_append(ctx, kv: tri_kv, k_new_ptr: int, v_new_ptr: int, pos_new_ptr: int, stream: int) -> int:
+    return _lib.tri_append(ctx, ctypes.byref(kv), k_new_ptr, v_new_ptr, pos_new_ptr, stream)
 
 
 def tri_get_error(ctx, stream: int):
@@ -254,6 +259,23 @@ class TriContext:
         st = tri_score(self.handle, kv, t.data_ptr(), _ptr(raw), _ptr(zmax), _stream_handle(stream))
         if check and st != TRI_OK:
             raise TriError(st, "tri_score", tri_last_error(self.handle))
+        return st
+
+    def append(self, K, V, pos, lens, block_table, K_new, V_new, pos_new, lens_out="inplace", n_pages=None,
+               layer_begin=0, stream=None, check=True):
+        """Append one token per sequence to a paged cache (see make_kv for the layouts):
+        K_new, V_new bf16 [n_layers][batch][n_kv_heads][head_dim], pos_new int32 [batch]."""
+        if isinstance(lens_out, str):
+            lens_out = lens
+        kv = make_kv(K, V, pos, lens, lens_out, block_table, n_pages=n_pages, layer_begin=layer_begin)
+        for name, x, dt in (("K_new", K_new, torch.bfloat16), ("V_new", V_new, torch.bfloat16),
+                            ("pos_new", pos_new, torch.int32)):
+            if x.dtype != dt or not x.is_cuda or not x.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous CUDA tensor of {dt}")
+        st = tri_append(self.handle, kv, K_new.data_ptr(), V_new.data_ptr(), pos_new.data_ptr(),
+                        _stream_handle(stream))
+        if check and st != TRI_OK:
+            raise TriError(st, "tri_append", tri_last_error(self.handle))
         return st
 
     def calibrate_estimate(self, Q, layout, out=None, stream=None, check=True):

@@ -1,0 +1,202 @@
+"""The decode loop around the prune: tri_append between prunes, a prune every C tokens, and the
+pages past each pruned length returned to a free list and reused.
+
+The page pool is tight, so freed pages come back into use. Before every prune the cache must
+hold exactly the rows expected (the previous prune's output plus every appended row, bit for
+bit); every prune is checked unit by unit against the fp64 oracle run on the rows it saw
+(kept set up to threshold ties, compacted rows bit-exact, lengths).
+"""
+import numpy as np
+import pytest
+import torch
+
+import tri_synth as ts
+import gpu_util as gu
+import oracle
+from rope_aware_key_tri_b200 import tri
+
+pytestmark = pytest.mark.gpu
+
+L, HKV, G, D, BATCH, PS, B, C = 2, 2, 4, 64, 3, 16, 48, 32
+MAX_PAGES = 8                 # capacity 128 slots per unit
+N_PAGES = 22                  # tight: a sequence holds at most ceil((B + C) / PS) = 5 pages at a prune
+PREFILL = (5, 37, 46)
+STEPS = 5 * C
+
+
+def _bits(x):
+    return x.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+class Pool:
+    """The caller's side of a paged cache: pools, block table and a FIFO free list of pages."""
+
+    def __init__(self, rng):
+        self.K = torch.from_numpy(rng.integers(0, 1 << 16, (L, N_PAGES, HKV, PS, D), dtype=np.uint16)
+                                  .view(np.int16)).view(torch.bfloat16).cuda()   # garbage, never read
+        self.V = self.K.clone()
+        self.P = torch.full((L, N_PAGES, HKV, PS), -7, dtype=torch.int32, device="cuda")
+        self.bt = np.full((BATCH, MAX_PAGES), -1, dtype=np.int32)
+        self.bt_dev = torch.from_numpy(self.bt).cuda()
+        self.free = list(range(N_PAGES))
+        self.reused = 0
+        self.handed = set()
+
+    def ensure(self, s, slot):
+        j = slot // PS
+        if self.bt[s, j] < 0:
+            p = self.free.pop(0)
+            if p in self.handed:
+                self.reused += 1
+            self.handed.add(p)
+            self.bt[s, j] = p
+
+    def reclaim(self, s, n):
+        for j in range((n + PS - 1) // PS, MAX_PAGES):
+            if self.bt[s, j] >= 0:
+                self.free.append(int(self.bt[s, j]))
+                self.bt[s, j] = -1
+
+    def sync(self):
+        self.bt_dev.copy_(torch.from_numpy(self.bt))
+
+    def rows(self, l, s, g, n):
+        slots = np.arange(n)
+        pages = torch.from_numpy(self.bt[s, slots // PS].astype(np.int64)).cuda()
+        offs = torch.from_numpy(slots % PS).cuda()
+        return (_bits(self.K[l, pages, g, offs]), _bits(self.V[l, pages, g, offs]),
+                self.P[l, pages, g, offs].cpu().numpy())
+
+
+def test_decode_loop_append_prune_reclaim():
+    rng = np.random.default_rng(11)
+    spec = ts.CacheSpec(name="loop", head_dim=D, group=G, n_kv_heads=HKV, n_layers=L, batch=BATCH,
+                        rope_base=1e4, budget=B, offsets=ts.pow2_offsets(10), positions="from_zero",
+                        lens=(1,) * BATCH, key_sigma=(0.3, 0.3), page_size=PS)
+    qm, qn, R, offsets = ts.make_stats(spec, 5)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(L, HKV, G, D, spec.rope_base, spec.layout, qm, qn, R, offsets)
+    pool = Pool(rng)
+    lens = np.zeros(BATCH, dtype=np.int64)
+    tpos = np.zeros(BATCH, dtype=np.int64)        # next position of each sequence
+    expect = {(l, s, g): [np.zeros((0, D), np.uint16), np.zeros((0, D), np.uint16), np.zeros(0, np.int32)]
+              for l in range(L) for s in range(BATCH) for g in range(HKV)}
+
+    def draw():
+        k = torch.from_numpy(rng.normal(0, 0.5, (L, BATCH, HKV, D)).astype(np.float32)).to(torch.bfloat16)
+        v = torch.from_numpy(rng.normal(0, 1.0, (L, BATCH, HKV, D)).astype(np.float32)).to(torch.bfloat16)
+        return k, v
+
+    # prefill through the same entry point: sequence s takes part once its turn comes, so the
+    # lengths end up ragged (PREFILL); a sequence outside its turn is refused by pointing its
+    # slot at an unallocated page, which also exercises the refusal path
+    for step in range(max(PREFILL)):
+        active = [s for s in range(BATCH) if max(PREFILL) - PREFILL[s] <= step]
+        for s in active:
+            pool.ensure(s, int(lens[s]))
+        pool.sync()
+        k, v = draw()
+        lens_dev = torch.from_numpy(lens.astype(np.int32)).cuda()
+        pos_new = torch.from_numpy(tpos.astype(np.int32)).cuda()
+        ctx.append(pool.K, pool.V, pool.P, lens_dev, pool.bt_dev, k.cuda(), v.cuda(), pos_new)
+        st, code, unit = ctx.get_error()
+        if len(active) < BATCH:
+            assert st == tri.TRI_EDEVICE and code == 2, (st, code)  # TRI_DEV_BAD_PAGE
+        else:
+            assert st == tri.TRI_OK, (st, code, unit)
+        new = lens_dev.cpu().numpy()
+        for s in range(BATCH):
+            if s in active:
+                assert new[s] == lens[s] + 1
+                for l in range(L):
+                    for g in range(HKV):
+                        e = expect[(l, s, g)]
+                        e[0] = np.vstack([e[0], _bits(k[l, s, g])[None]])
+                        e[1] = np.vstack([e[1], _bits(v[l, s, g])[None]])
+                        e[2] = np.append(e[2], np.int32(tpos[s]))
+                tpos[s] += 1
+            else:
+                assert new[s] == lens[s]
+        lens = new.astype(np.int64)
+    assert tuple(lens) == PREFILL
+
+    prunes = 0
+    for step in range(STEPS):
+        for s in range(BATCH):
+            pool.ensure(s, int(lens[s]))
+        pool.sync()
+        k, v = draw()
+        lens_dev = torch.from_numpy(lens.astype(np.int32)).cuda()
+        ctx.append(pool.K, pool.V, pool.P, lens_dev, pool.bt_dev, k.cuda(), v.cuda(),
+                   torch.from_numpy(tpos.astype(np.int32)).cuda())
+        assert ctx.get_error()[0] == tri.TRI_OK
+        assert np.array_equal(lens_dev.cpu().numpy(), lens + 1)
+        for l in range(L):
+            for s in range(BATCH):
+                for g in range(HKV):
+                    e = expect[(l, s, g)]
+                    e[0] = np.vstack([e[0], _bits(k[l, s, g])[None]])
+                    e[1] = np.vstack([e[1], _bits(v[l, s, g])[None]])
+                    e[2] = np.append(e[2], np.int32(tpos[s]))
+        lens += 1
+        tpos += 1
+        if (step + 1) % C:
+            continue
+        # ---- a prune: the cache holds exactly what was appended since the last one ----------
+        pre = {}
+        for (l, s, g), e in expect.items():
+            got = pool.rows(l, s, g, int(lens[s]))
+            assert np.array_equal(got[0], e[0]) and np.array_equal(got[1], e[1]) and np.array_equal(got[2], e[2]), \
+                f"step {step}: unit {(l, s, g)} does not hold the appended rows"
+            pre[(l, s, g)] = got
+        lens_dev = torch.from_numpy(lens.astype(np.int32)).cuda()
+        t_dev = torch.from_numpy(tpos.astype(np.int32)).cuda()
+        ctx.prune(pool.K, pool.V, pool.P, lens_dev, t_dev, B, block_table=pool.bt_dev)
+        assert ctx.get_error()[0] == tri.TRI_OK
+        new = lens_dev.cpu().numpy().astype(np.int64)
+        assert np.array_equal(new, np.minimum(lens, B))
+        for (l, s, g), (kb, vb, pb) in pre.items():
+            n, m = int(lens[s]), int(new[s])
+            out = pool.rows(l, s, g, m)
+            if n > B:
+                h0 = g * G
+                orc = oracle.prune_unit(kb, vb, pb, int(tpos[s]), qm[l, h0:h0 + G], qn[l, h0:h0 + G],
+                                        R[l, h0:h0 + G], offsets, spec.rope_base, B, spec.layout)
+                kept = gu.kept_from_output(pb, out[2])
+                gu.check_kept(kept, orc, B, f"prune {prunes} unit {(l, s, g)}")
+                gu.check_compacted((kb, vb, pb), out, kept, f"prune {prunes} unit {(l, s, g)}")
+            else:
+                assert np.array_equal(out[0], kb[:m]) and np.array_equal(out[2], pb[:m])
+            expect[(l, s, g)] = [out[0], out[1], out[2]]
+        lens = new
+        for s in range(BATCH):
+            pool.reclaim(s, int(lens[s]))
+        pool.sync()
+        prunes += 1
+    assert prunes == STEPS // C
+    assert pool.reused > 0, "the tight pool never handed a freed page out again"
+    ctx.close()
+
+
+def test_append_refuses_full_sequences():
+    spec = ts.CacheSpec(name="full", head_dim=128, group=2, n_kv_heads=1, n_layers=1, batch=2,
+                        rope_base=1e4, budget=16, offsets=(1, 2), positions="from_zero", lens=(1, 1),
+                        page_size=16)
+    qm, qn, R, offsets = ts.make_stats(spec, 1)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(1, 1, 2, 128, 1e4, spec.layout, qm, qn, R, offsets)
+    K = torch.zeros((1, 2, 1, 16, 128), dtype=torch.bfloat16, device="cuda")
+    V = torch.zeros_like(K)
+    P = torch.zeros((1, 2, 1, 16), dtype=torch.int32, device="cuda")
+    bt = torch.tensor([[0], [1]], dtype=torch.int32, device="cuda")   # one page each: capacity 16
+    lens = torch.tensor([16, 3], dtype=torch.int32, device="cuda")     # sequence 0 is full
+    kn = torch.ones((1, 2, 1, 128), dtype=torch.bfloat16, device="cuda")
+    ctx.append(K, V, P, lens, bt, kn, kn, torch.tensor([16, 3], dtype=torch.int32, device="cuda"))
+    st, code, unit = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == 1  # TRI_DEV_LEN_GT_CAP
+    assert lens.cpu().tolist() == [16, 4]
+    assert torch.all(K[0, 1, 0, 3] == 1) and int(P[0, 1, 0, 3]) == 3
+    assert torch.all(K[0, 0] == 0)
+    # host check: a dense cache (no block table) is rejected before anything is launched
+    assert ctx.append(K, V, P, lens, None, kn, kn, lens, check=False) == tri.TRI_EINVAL
+    ctx.close()
