@@ -705,7 +705,8 @@ def main():
                    "group": spec.group, "head_dim": spec.head_dim, "batch_per_gpu": spec.batch,
                    "keys_per_unit": sorted(set(int(x) for x in res["lens"]))[:4],
                    "budget": spec.budget, "parallelism": f"replicas x{world} (sequence shards, no collective)",
-                   "l2": "256 MiB buffer written between steps; 19 GB of inputs > L2",
+                   "l2": "256 MiB buffer written between steps (flushes L2); K+V inputs %.2f GB"
+                         % ((cache.K.numel() + cache.V.numel()) * 2 / 1e9),
                    "timed": "CUDA events around the tri_prune launch; row restore between steps untimed"},
         "roofline": res["roofline"],
         "clocks": res["clocks"],
