@@ -200,3 +200,49 @@ def test_append_refuses_full_sequences():
     # host check: a dense cache (no block table) is rejected before anything is launched
     assert ctx.append(K, V, P, lens, None, kn, kn, lens, check=False) == tri.TRI_EINVAL
     ctx.close()
+
+
+def test_append_replays_from_a_cuda_graph():
+    # the appends of a page span captured once and replayed give the same cache as the same
+    # appends issued one by one
+    spec = ts.CacheSpec(name="graph", head_dim=128, group=4, n_kv_heads=2, n_layers=2, batch=3,
+                        rope_base=1e4, budget=16, offsets=(1, 2), positions="from_zero", lens=(1, 1, 1),
+                        page_size=16)
+    qm, qn, R, offsets = ts.make_stats(spec, 2)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(2, 2, 4, 128, 1e4, spec.layout, qm, qn, R, offsets)
+    steps = 16
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    new_k = torch.randn((steps, 2, 3, 2, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    new_v = torch.randn((steps, 2, 3, 2, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    bt = torch.tensor([[0, 1], [2, 3], [4, 5]], dtype=torch.int32, device="cuda")
+
+    def fresh():
+        K = torch.zeros((2, 6, 2, 16, 128), dtype=torch.bfloat16, device="cuda")
+        return K, K.clone(), torch.full((2, 6, 2, 16), -1, dtype=torch.int32, device="cuda"), \
+            torch.tensor([16, 16, 16], dtype=torch.int32, device="cuda"), \
+            torch.tensor([40, 50, 60], dtype=torch.int32, device="cuda")
+
+    K1, V1, P1, l1, t1 = fresh()
+    for i in range(steps):
+        ctx.append(K1, V1, P1, l1, bt, new_k[i], new_v[i], t1)
+        t1.add_(1)
+    K2, V2, P2, l2, t2 = fresh()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        for i in range(steps):
+            ctx.append(K2, V2, P2, l2, bt, new_k[i], new_v[i], t2)
+            t2.add_(1)
+    torch.cuda.current_stream().wait_stream(side)
+    assert l2.cpu().tolist() == [16, 16, 16]  # capturing ran nothing
+    g.replay()
+    torch.cuda.synchronize()
+    assert ctx.get_error()[0] == tri.TRI_OK
+    assert l1.cpu().tolist() == l2.cpu().tolist() == [32, 32, 32]
+    assert torch.equal(K1.view(torch.int16), K2.view(torch.int16))
+    assert torch.equal(V1.view(torch.int16), V2.view(torch.int16))
+    assert torch.equal(P1, P2) and torch.equal(t1, t2)
+    assert int(P1[0, 1, 0, 0]) == 40 and int(P1[1, 5, 1, 15]) == 75
+    ctx.close()
