@@ -49,6 +49,8 @@ def _bind(L):
     L.tri_oracle_prune_batch.argtypes = [i32, i32, i32, i32, i32, i32, f64, P, i32, P,
                                          P, P, P, P, P, P, P, P, P, i32]
     L.tri_oracle_prune_batch.restype = i32
+    L.tri_oracle_unit_scores_max.argtypes = L.tri_oracle_unit_scores.argtypes
+    L.tri_oracle_unit_scores_max.restype = i32
     L.tri_oracle_calibrate.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
     L.tri_oracle_calibrate.restype = i32
     return L
@@ -62,13 +64,15 @@ def _p(a):
     return a.ctypes.data_as(ctypes.c_void_p) if a is not None else None
 
 
-def unit_scores(K_bits, pos, t, q_mean, q_norm, R, offsets, base, layout=HALF, L=None):
+def unit_scores(K_bits, pos, t, q_mean, q_norm, R, offsets, base, layout=HALF, L=None, combine="mean"):
     """Per-head scores of one unit: returns (s, trig, norm), each fp64 [G][N].
 
     K_bits: uint16 [N][d] bf16 bits of the stored keys; pos: int [N];
-    q_mean: [G][d]; q_norm, R: [G][d/2]; offsets: the future-offset set.
+    q_mean: [G][d]; q_norm, R: [G][d/2]; offsets: the future-offset set;
+    combine: "mean" (the pass) or "max" over the offsets (the variant).
     """
     L = L or lib()
+    fn = {"mean": L.tri_oracle_unit_scores, "max": L.tri_oracle_unit_scores_max}[combine]
     K_bits = _c(K_bits, np.uint16)
     N, d = K_bits.shape
     q_mean = _c(q_mean, np.float32).reshape(-1, d)
@@ -78,9 +82,9 @@ def unit_scores(K_bits, pos, t, q_mean, q_norm, R, offsets, base, layout=HALF, L
     pos = _c(pos, np.int32)
     off = _c(offsets, np.int64)
     s = np.empty((G, N)); tr = np.empty((G, N)); nm = np.empty((G, N))
-    rc = L.tri_oracle_unit_scores(d, G, layout, float(base), _p(off), len(off), int(t),
-                                  _p(q_mean), _p(q_norm), _p(R), _p(K_bits), _p(pos), N,
-                                  _p(s), _p(tr), _p(nm))
+    rc = fn(d, G, layout, float(base), _p(off), len(off), int(t),
+            _p(q_mean), _p(q_norm), _p(R), _p(K_bits), _p(pos), N,
+            _p(s), _p(tr), _p(nm))
     if rc != 0:
         raise ValueError("tri_oracle_unit_scores rejected its arguments")
     return s, tr, nm

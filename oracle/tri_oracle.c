@@ -97,11 +97,14 @@ int tri_oracle_version(void) { return 1; }
  * Outputs s [G][N] (and optionally the two terms separately).
  * Returns 0, or -1 on bad arguments.
  */
-int tri_oracle_unit_scores(int d, int G, int layout, double base,
-                           const int64_t *offsets, int n_off, int64_t t,
-                           const float *q_mean, const float *q_norm, const float *R,
-                           const uint16_t *K, const int32_t *pos, int N,
-                           double *s_out, double *trig_out, double *norm_out)
+#define TRI_ORACLE_MEAN_OVER_DELTA 0
+#define TRI_ORACLE_MAX_OVER_DELTA 1
+
+static int unit_scores(int combine, int d, int G, int layout, double base,
+                       const int64_t *offsets, int n_off, int64_t t,
+                       const float *q_mean, const float *q_norm, const float *R,
+                       const uint16_t *K, const int32_t *pos, int N,
+                       double *s_out, double *trig_out, double *norm_out)
 {
     if (d < 2 || (d & 1) || G < 1 || N < 0 || n_off < 1 || !offsets || !s_out)
         return -1;
@@ -142,7 +145,7 @@ int tri_oracle_unit_scores(int d, int G, int layout, double base,
             karg[f] = atan2(pi, pr);
         }
         for (int h = 0; h < G; ++h) {
-            double trig = 0.0;
+            double trig = 0.0, best = 0.0;
             for (int j = 0; j < n_off; ++j) {
                 const double delta = (double)((int64_t)t + offsets[j]) - p;
                 double series = 0.0;
@@ -151,8 +154,10 @@ int tri_oracle_unit_scores(int d, int G, int layout, double base,
                     series += qmag[h * F + f] * kmag[f] * cos(omega[f] * delta + phi);
                 }
                 trig += series;
+                if (j == 0 || series > best) best = series;
             }
             trig /= (double)n_off;
+            if (combine == TRI_ORACLE_MAX_OVER_DELTA) trig = best;
             double norm = 0.0;
             for (int f = 0; f < F; ++f)
                 norm += (1.0 - (double)R[h * F + f]) * (double)q_norm[h * F + f] * kmag[f];
@@ -163,6 +168,32 @@ int tri_oracle_unit_scores(int d, int G, int layout, double base,
     }
     free(omega); free(qmag); free(qarg); free(kmag); free(karg);
     return 0;
+}
+
+int tri_oracle_unit_scores(int d, int G, int layout, double base,
+                           const int64_t *offsets, int n_off, int64_t t,
+                           const float *q_mean, const float *q_norm, const float *R,
+                           const uint16_t *K, const int32_t *pos, int N,
+                           double *s_out, double *trig_out, double *norm_out)
+{
+    return unit_scores(TRI_ORACLE_MEAN_OVER_DELTA, d, G, layout, base, offsets, n_off, t, q_mean, q_norm, R,
+                       K, pos, N, s_out, trig_out, norm_out);
+}
+
+/*
+ * The same scores with the offsets combined by the maximum instead of the mean: the
+ * trigonometric term is max over delta of S_trig(k, t + delta - p), the reading of
+ * [Deep-dive] §3.3 and of the listing of its §4.2 (where the norm score is then added).
+ * The pass built on the GPU uses the mean; this mode is the definition for a variant.
+ */
+int tri_oracle_unit_scores_max(int d, int G, int layout, double base,
+                               const int64_t *offsets, int n_off, int64_t t,
+                               const float *q_mean, const float *q_norm, const float *R,
+                               const uint16_t *K, const int32_t *pos, int N,
+                               double *s_out, double *trig_out, double *norm_out)
+{
+    return unit_scores(TRI_ORACLE_MAX_OVER_DELTA, d, G, layout, base, offsets, n_off, t, q_mean, q_norm, R,
+                       K, pos, N, s_out, trig_out, norm_out);
 }
 
 /*

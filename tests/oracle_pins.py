@@ -252,6 +252,42 @@ def pin_compaction(L, seed=7):
             assert r["zmax"][kept].min() >= r["zmax"][drop].max()
 
 
+def pin_max_over_delta(L, seed=9):
+    """The variant that combines the offsets by the maximum: with R = 1 it equals max over delta
+    of the textbook-RoPE dot product; with one offset it equals the mean mode; it is never below
+    the mean mode; the norm term is the same in both modes; positions still cancel."""
+    rng = np.random.default_rng(seed)
+    for d, base, offsets in ((8, 1e4, [1, 2]), (64, 1e4, [1 << i for i in range(11)]),
+                             (128, 1e6, [1 << i for i in range(17)])):
+        for layout in (oracle.HALF, oracle.INTERLEAVED):
+            G, N = 3, 17
+            q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base, r_one=True)
+            s, trig, norm = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets, base, layout, L=L,
+                                               combine="max")
+            kval = _bf16_value(K)
+            want = np.full((G, N), -np.inf)
+            for h in range(G):
+                for dl in offsets:
+                    want[h] = np.maximum(want[h], kval @ rope_rotate(q_mean[h], t + dl, base, layout))
+            scale = np.abs(want).max()
+            assert np.abs(norm).max() == 0.0
+            assert np.abs(s - want).max() <= 1e-9 * scale, (d, layout, np.abs(s - want).max(), scale)
+            # R < 1: max >= mean, identical norm terms, one offset gives the mean mode exactly
+            q_mean, q_norm, R, K, pos, t = _rand_unit(rng, d, G, N, layout, base)
+            s_mx, tr_mx, nm_mx = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets, base, layout, L=L,
+                                                    combine="max")
+            s_mn, tr_mn, nm_mn = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets, base, layout, L=L)
+            assert np.all(tr_mx >= tr_mn - 1e-12 * np.abs(tr_mn).max())
+            assert np.array_equal(nm_mx, nm_mn)
+            one = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets[-1:], base, layout, L=L, combine="max")
+            one_mean = oracle.unit_scores(K, pos, t, q_mean, q_norm, R, offsets[-1:], base, layout, L=L)
+            assert np.array_equal(one[0], one_mean[0])
+            # positions cancel: the same stored keys at other positions, same t
+            pos2 = np.sort(rng.choice(int(pos[-1]) + 1, N, replace=False)).astype(np.int32)
+            s2 = oracle.unit_scores(K, pos2, t, q_mean, q_norm, R, offsets, base, layout, L=L, combine="max")[0]
+            assert np.abs(s2 - s_mx).max() <= 1e-9 * np.abs(s_mx).max()
+
+
 def _calib_tokens(bands, d, layout):
     """[T][d] real vectors from [T][F][2] band samples, in the given rotary layout."""
     bands = np.asarray(bands, dtype=np.float64)
@@ -335,4 +371,5 @@ def pin_calibrate_invariants(L, seed=8):
 ALL_PINS = [pin_hand_examples, pin_rope_dot_closed_form, pin_positions_cancel,
             pin_t_shift_is_query_rotation, pin_norm_rotation_invariant_and_linear,
             pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction,
-            pin_calibrate_hand_example, pin_calibrate_closed_forms, pin_calibrate_invariants]
+            pin_calibrate_hand_example, pin_calibrate_closed_forms, pin_calibrate_invariants,
+            pin_max_over_delta]

@@ -30,6 +30,8 @@ MUTANTS = {
     "qmag_not_kmag": ("series += qmag[h * F + f] * kmag[f] *", "series += qmag[h * F + f] *"),
     "flat_head_not_zero": ("const int flat = !(hi > lo);", "const int flat = 0;"),
     "no_resort": ("qsort(kept_out, (size_t)M, sizeof(int32_t), idx_cmp);", ""),
+    "max_mode_takes_min": ("if (j == 0 || series > best) best = series;", "if (j == 0 || series < best) best = series;"),
+    "max_mode_keeps_mean": ("if (combine == TRI_ORACLE_MAX_OVER_DELTA) trig = best;", ""),
     "calib_R_inverted": ("mm > 0.0 ? sqrt(mr * mr + mi * mi) / mm : 0.0;", "mm > 0.0 ? mm / sqrt(mr * mr + mi * mi) : 0.0;"),
     "calib_squared_modulus": ("sm += sqrt(re * re + im * im);", "sm += re * re + im * im;"),
     "calib_sum_not_mean": ("const double mr = sr / (double)T, mi = si / (double)T, mm = sm / (double)T;",
