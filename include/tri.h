@@ -157,8 +157,9 @@ TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads
  * caller (an id in [0, n_pages)); freeing the pages past a sequence's length after a prune
  * is the caller's business too. A sequence whose slot is past its capacity or lands in an
  * unallocated page is refused as a whole (lens_out[s] = lens[s]; tri_get_error reports
- * TRI_DEV_LEN_GT_CAP or TRI_DEV_BAD_PAGE); a refused sequence may have received the rows of
- * some layers before the refusal. Needs the statistics loaded (for n_kv_heads and head_dim).
+ * TRI_DEV_LEN_GT_CAP or TRI_DEV_BAD_PAGE): every unit of a sequence sees the same slot and
+ * page, so a refused sequence receives no row. Needs the statistics loaded (for n_kv_heads
+ * and head_dim).
  * Two launches on `stream`.
  */
 TRI_API tri_status tri_append(tri_ctx *ctx, const tri_kv *kv, const void *K_new, const void *V_new,
