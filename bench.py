@@ -204,6 +204,8 @@ def run_ours(args, rank, world, dist_mod):
                        cache.q_mean, cache.q_norm_mean, cache.R, cache.offsets)
     if args.cluster_size or args.buffers:
         ctx.set_tuning(args.cluster_size, args.buffers)
+    if args.combine != "mean":
+        ctx.set_offset_combine(args.combine)
     lens_host = cache.lens_host.tolist()
     lens0 = cache.lens.clone()
     paged = cache.paged
@@ -275,6 +277,10 @@ def run_ours(args, rank, world, dist_mod):
     keys_rank = sum(lens_host) * spec.n_layers * spec.n_kv_heads
     keys_total = keys_rank * world
     value = keys_total / (mean_ms_max / 1e3)
+    # max mode: prefix + phase kernels, then per chunk of layers (scores under 1 GiB) the
+    # coefficient images, the tensor-core scoring and the fused select/compaction (+ a memset)
+    per_layer_scores = spec.batch * spec.n_kv_heads * cache.cap * spec.group * 4
+    n_chunks = -(-spec.n_layers // max(1, min(spec.n_layers, (1 << 30) // per_layer_scores)))
     abytes = algorithmic_bytes(lens_host, spec.n_layers, spec.n_kv_heads, spec.head_dim, B)
     peak, peak_kind = measured_peak()
     achieved = abytes / (mean_ms / 1e3) / 1e9
@@ -287,7 +293,7 @@ def run_ours(args, rank, world, dist_mod):
                      "frac": achieved / peak, "traffic": ncu_traffic(args.workload),
                      "algorithmic_bytes": abytes, "peak_kind": f"{peak_kind} (burst copy)"},
         "clocks": clk.summary(),
-        "gpu_launches": args.steps,
+        "gpu_launches": args.steps * (1 if args.combine == "mean" else 2 + 3 * n_chunks),
         "keys_per_rank": keys_rank,
         "lens": lens_host,
     }
@@ -386,7 +392,7 @@ def oracle_sample(cache, spec, n_units, trunc=None):
     return ids, Kb, Pb, np.array(n_keys, np.int32), tt, qm, qn, RR
 
 
-def time_oracle(cache, spec, budget_s=10.0, cores=None, min_steps=1):
+def time_oracle(cache, spec, budget_s=10.0, cores=None, min_steps=1, combine="mean"):
     """Run the oracle on a bounded sample; returns (keys/s, cores, description)."""
     import numpy as np
 
@@ -396,7 +402,8 @@ def time_oracle(cache, spec, budget_s=10.0, cores=None, min_steps=1):
     ids, Kb, Pb, nk, tt, qm, qn, RR = oracle_sample(cache, spec, 1, trunc=1024)
     t0 = time.perf_counter()
     oracle.prune_batch(Kb, Pb, nk, tt, qm, qn, RR, cache.offsets, spec.rope_base,
-                       max(1, spec.budget * 1024 // max(1, int(cache.lens_host.max()))), spec.layout, n_threads=1)
+                       max(1, spec.budget * 1024 // max(1, int(cache.lens_host.max()))), spec.layout, n_threads=1,
+                       combine=combine)
     per_key = (time.perf_counter() - t0) / 1024.0
     N = int(cache.lens_host.max())
     unit_s = per_key * N
@@ -411,7 +418,7 @@ def time_oracle(cache, spec, budget_s=10.0, cores=None, min_steps=1):
     Bs = spec.budget if trunc is None else max(1, spec.budget * trunc // N)
     t0 = time.perf_counter()
     oracle.prune_batch(Kb, Pb, nk, tt, qm, qn, RR, cache.offsets, spec.rope_base, Bs, spec.layout,
-                       n_threads=cores)
+                       n_threads=cores, combine=combine)
     el = time.perf_counter() - t0
     keys = int(nk.sum())
     what = f"{len(ids)} of {cache.n_units} units" + (
@@ -699,6 +706,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0,
                     help="override the workload's layer count (smaller cases for profiling)")
     ap.add_argument("--cluster-size", type=int, default=0)
+    ap.add_argument("--combine", default="mean", choices=["mean", "max"],
+                    help="how the future offsets combine in the score (max: the tensor-core variant)")
     ap.add_argument("--buffers", type=int, default=0)
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
@@ -754,7 +763,8 @@ def main():
                    "budget": spec.budget, "parallelism": f"replicas x{world} (sequence shards, no collective)",
                    "l2": "256 MiB buffer written between steps (flushes L2); K+V inputs %.2f GB"
                          % ((cache.K.numel() + cache.V.numel()) * 2 / 1e9),
-                   "timed": "CUDA events around the tri_prune launch; row restore between steps untimed"},
+                   "offsets_combine": args.combine,
+                   "timed": "CUDA events around the tri_prune call; row restore between steps untimed"},
         "roofline": res["roofline"],
         "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"],
@@ -764,7 +774,7 @@ def main():
     if "e2e" in res:
         out["e2e"] = res["e2e"]
     if rank == 0 and world == 1 and not args.no_cpu:
-        v, cores, what = time_oracle(cache, spec, budget_s=10.0)
+        v, cores, what = time_oracle(cache, spec, budget_s=10.0, combine=args.combine)
         out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": what}
     if rank == 0:
         print(json.dumps(out), flush=True)

@@ -71,6 +71,12 @@ typedef enum {
     TRI_ROPE_INTERLEAVED = 1  /* band f = dims (2f, 2f + 1): GPT-J rotary layout */
 } tri_rope_layout;
 
+/* How the future offsets delta combine in the trigonometric score (tri_set_offset_combine). */
+typedef enum {
+    TRI_OFFSETS_MEAN = 0,  /* mean over delta (default): folds into one coefficient per band */
+    TRI_OFFSETS_MAX = 1    /* max over delta ([Deep-dive] §3.3 and its §4.2 scoring code) */
+} tri_offset_combine;
+
 /* Device-side problem codes reported by tri_get_error in *detail_code. */
 enum {
     TRI_DEV_NONE = 0,
@@ -253,6 +259,30 @@ TRI_API tri_status tri_get_error(tri_ctx *ctx, void *stream, int32_t *detail_cod
  * return TRI_EUNSUPPORTED.
  */
 TRI_API tri_status tri_set_tuning(tri_ctx *ctx, int cluster_size, int buffers_per_warp);
+
+/*
+ * Choose how later tri_prune / tri_score calls on this context combine the future offsets.
+ *   TRI_OFFSETS_MEAN  s_h = mean over delta of S_trig + S_norm. The mean folds into one
+ *                     complex coefficient per band (A_f), so a key costs one dot product per
+ *                     head. The default.
+ *   TRI_OFFSETS_MAX   s_h = max over delta of S_trig + S_norm: the reading of [Deep-dive] §3.3
+ *                     (score at every offset of the geometric set, keep the largest) and of
+ *                     its §4.2 scoring code, which then adds the norm score. This does not
+ *                     fold: every key needs group * n_offsets dot products, run as a
+ *                     tensor-core contraction (the bf16 keys against a hi + lo bf16 split of
+ *                     the fp64 coefficients qbar_f e^{i omega_f (t + delta)}, fp32
+ *                     accumulation), followed by the same z-score, max over the group,
+ *                     top-B select and compaction.
+ * Everything else (arguments, results, in-place semantics, device status codes) is the same
+ * in both modes. The max mode needs group * n_offsets <= 256 (else the call returns
+ * TRI_EUNSUPPORTED) and scratch that tri_prune / tri_score grow on demand: the scores of up
+ * to 1 GiB worth of layers at a time (n_layers_chunk * batch * n_kv_heads * cap_u * group * 4
+ * bytes; longer calls run in chunks of layers), one coefficient image per unit of a chunk
+ * (42 KB at head_dim 128, group 4, 17 offsets) and small tables. tri_prune_noalloc supports
+ * the mean only (TRI_EUNSUPPORTED in max mode). Errors: TRI_EINVAL (NULL context, unknown
+ * mode).
+ */
+TRI_API tri_status tri_set_offset_combine(tri_ctx *ctx, int combine);
 
 /* Text of the last host-side failure on this context (the CUDA error and the call that
  * returned it), or an empty string. Valid until the next call on the context. */

@@ -49,6 +49,8 @@ def _bind(L):
     L.tri_oracle_prune_batch.argtypes = [i32, i32, i32, i32, i32, i32, f64, P, i32, P,
                                          P, P, P, P, P, P, P, P, P, i32]
     L.tri_oracle_prune_batch.restype = i32
+    L.tri_oracle_prune_batch_max.argtypes = L.tri_oracle_prune_batch.argtypes
+    L.tri_oracle_prune_batch_max.restype = i32
     L.tri_oracle_unit_scores_max.argtypes = L.tri_oracle_unit_scores.argtypes
     L.tri_oracle_unit_scores_max.restype = i32
     L.tri_oracle_calibrate.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
@@ -128,9 +130,11 @@ def compact(kept, K_bits, V_bits, pos, L=None):
     return Ko, Vo, po
 
 
-def prune_unit(K_bits, V_bits, pos, t, q_mean, q_norm, R, offsets, base, B, layout=HALF, L=None):
-    """The whole pass on one unit. Returns a dict with s, z, zmax, kept and the compacted rows."""
-    s, tr, nm = unit_scores(K_bits, pos, t, q_mean, q_norm, R, offsets, base, layout, L)
+def prune_unit(K_bits, V_bits, pos, t, q_mean, q_norm, R, offsets, base, B, layout=HALF, L=None,
+               combine="mean"):
+    """The whole pass on one unit. Returns a dict with s, z, zmax, kept and the compacted rows.
+    combine: how the offsets combine in the trigonometric score ("mean" or "max")."""
+    s, tr, nm = unit_scores(K_bits, pos, t, q_mean, q_norm, R, offsets, base, layout, L, combine=combine)
     z, zm = zmax(s, L)
     kept = select(zm, B, L)
     Ko, Vo, po = compact(kept, K_bits, V_bits, pos, L)
@@ -138,8 +142,8 @@ def prune_unit(K_bits, V_bits, pos, t, q_mean, q_norm, R, offsets, base, B, layo
 
 
 def prune_batch(K_bits, pos, lens, t, q_mean, q_norm, R, offsets, base, B, layout=HALF,
-                n_threads=0, want_zmax=False, L=None):
-    """Selection for many units at once (threads over units).
+                n_threads=0, want_zmax=False, L=None, combine="mean"):
+    """Selection for many units at once (threads over units); combine "mean" or "max".
 
     K_bits [U][S][d] uint16, pos [U][S], lens [U], t [U], q_mean [U][G][d],
     q_norm/R [U][G][d/2]. Returns (kept [U][B] int32, n_kept [U], zmax or None).
@@ -154,9 +158,10 @@ def prune_batch(K_bits, pos, lens, t, q_mean, q_norm, R, offsets, base, B, layou
     off = _c(offsets, np.int64)
     kept = np.zeros((U, B), np.int32); nk = np.zeros(U, np.int32)
     zm = np.zeros((U, S)) if want_zmax else None
-    rc = L.tri_oracle_prune_batch(U, S, int(B), d, G, layout, float(base), _p(off), len(off), _p(t),
-                                  _p(q_mean), _p(q_norm), _p(R), _p(K_bits), _p(pos), _p(lens),
-                                  _p(zm), _p(kept), _p(nk), int(n_threads))
+    fn = {"mean": L.tri_oracle_prune_batch, "max": L.tri_oracle_prune_batch_max}[combine]
+    rc = fn(U, S, int(B), d, G, layout, float(base), _p(off), len(off), _p(t),
+            _p(q_mean), _p(q_norm), _p(R), _p(K_bits), _p(pos), _p(lens),
+            _p(zm), _p(kept), _p(nk), int(n_threads))
     if rc != 0:
         raise ValueError("tri_oracle_prune_batch rejected its arguments")
     return kept, nk, zm

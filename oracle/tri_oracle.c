@@ -301,12 +301,12 @@ int tri_oracle_compact(int d, int M, const int32_t *kept,
  * Outputs (optional where marked): zmax [n_units][stride] (NULL ok),
  * kept [n_units][B], n_kept [n_units]. Returns 0, or -1 on a bad argument.
  */
-int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int layout, double base,
-                           const int64_t *offsets, int n_off, const int64_t *t,
-                           const float *q_mean, const float *q_norm, const float *R,
-                           const uint16_t *K, const int32_t *pos, const int32_t *lens,
-                           double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
-                           int n_threads)
+static int prune_batch(int combine, int n_units, int stride, int B, int d, int G, int layout, double base,
+                       const int64_t *offsets, int n_off, const int64_t *t,
+                       const float *q_mean, const float *q_norm, const float *R,
+                       const uint16_t *K, const int32_t *pos, const int32_t *lens,
+                       double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                       int n_threads)
 {
     if (n_units < 0 || stride < 0 || B < 1 || d < 2 || G < 1)
         return -1;
@@ -322,10 +322,10 @@ int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int lay
         double *s = (double *)malloc(sizeof(double) * (size_t)G * (N > 0 ? N : 1));
         double *zm = (double *)malloc(sizeof(double) * (size_t)(N > 0 ? N : 1));
         if (!s || !zm) { free(s); free(zm); bad |= 1; continue; }
-        int rc = tri_oracle_unit_scores(d, G, layout, base, offsets, n_off, t[u],
-                                        q_mean + (size_t)u * G * d, q_norm + (size_t)u * G * F,
-                                        R + (size_t)u * G * F, K + (size_t)u * stride * d,
-                                        pos + (size_t)u * stride, N, s, NULL, NULL);
+        int rc = unit_scores(combine, d, G, layout, base, offsets, n_off, t[u],
+                             q_mean + (size_t)u * G * d, q_norm + (size_t)u * G * F,
+                             R + (size_t)u * G * F, K + (size_t)u * stride * d,
+                             pos + (size_t)u * stride, N, s, NULL, NULL);
         if (rc == 0) rc = tri_oracle_zmax(G, N, s, NULL, zm);
         if (rc == 0) {
             if (zmax_out) memcpy(zmax_out + (size_t)u * stride, zm, sizeof(double) * N);
@@ -337,6 +337,29 @@ int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int lay
         free(s); free(zm);
     }
     return bad ? -1 : 0;
+}
+
+int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int layout, double base,
+                           const int64_t *offsets, int n_off, const int64_t *t,
+                           const float *q_mean, const float *q_norm, const float *R,
+                           const uint16_t *K, const int32_t *pos, const int32_t *lens,
+                           double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                           int n_threads)
+{
+    return prune_batch(TRI_ORACLE_MEAN_OVER_DELTA, n_units, stride, B, d, G, layout, base, offsets, n_off, t,
+                       q_mean, q_norm, R, K, pos, lens, zmax_out, kept_out, n_kept_out, n_threads);
+}
+
+/* The same selection with the offsets combined by the maximum (tri_oracle_unit_scores_max). */
+int tri_oracle_prune_batch_max(int n_units, int stride, int B, int d, int G, int layout, double base,
+                               const int64_t *offsets, int n_off, const int64_t *t,
+                               const float *q_mean, const float *q_norm, const float *R,
+                               const uint16_t *K, const int32_t *pos, const int32_t *lens,
+                               double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                               int n_threads)
+{
+    return prune_batch(TRI_ORACLE_MAX_OVER_DELTA, n_units, stride, B, d, G, layout, base, offsets, n_off, t,
+                       q_mean, q_norm, R, K, pos, lens, zmax_out, kept_out, n_kept_out, n_threads);
 }
 
 /*

@@ -7,6 +7,8 @@
 // (the phase e^{i omega_f t} in fp64) so that a call never waits on the host.
 //
 //   [Deep-dive]  "TriAttention深度解析：用三角函数革命性压缩KV Cache，让长推理从「显存地狱」中脱困"
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -21,6 +23,7 @@
 #include "tri_kernel.cuh"
 #include "tri_calib.cuh"
 #include "tri_append.cuh"
+#include "tri_maxdelta.cuh"
 
 struct tri_ctx {
     int device = -1;
@@ -32,6 +35,21 @@ struct tri_ctx {
     double *d_omega = nullptr;
     double2 *d_Qc = nullptr;
     float *d_w = nullptr;
+    double2 *d_qbar = nullptr;      // [L][Hq][F] qbar itself (the max-over-offsets mode)
+    int64_t *d_offsets = nullptr;   // [n_off]
+    int n_off = 0;
+    int combine = TRI_OFFSETS_MEAN;
+    // scratch of the max-over-offsets mode, grown on demand
+    float *d_pre = nullptr;
+    size_t pre_bytes = 0;
+    unsigned char *d_image = nullptr;
+    size_t image_bytes = 0;
+    double2 *d_phase = nullptr;
+    size_t phase_bytes = 0;
+    int32_t *d_tile_prefix = nullptr;
+    size_t tile_prefix_bytes = 0;
+    int32_t *d_unit_fail = nullptr;
+    size_t unit_fail_bytes = 0;
     // device bookkeeping
     unsigned long long *d_status = nullptr;
     unsigned int *d_counter = nullptr;
@@ -83,10 +101,43 @@ void free_stats(tri_ctx *c) {
     cudaFree(c->d_omega);
     cudaFree(c->d_Qc);
     cudaFree(c->d_w);
+    cudaFree(c->d_qbar);
+    cudaFree(c->d_offsets);
     c->d_omega = nullptr;
     c->d_Qc = nullptr;
     c->d_w = nullptr;
+    c->d_qbar = nullptr;
+    c->d_offsets = nullptr;
+    c->n_off = 0;
     c->loaded = false;
+}
+
+// The fused kernel reading precomputed scores (the rotary layout plays no part there).
+KernelFn pick_pre_kernel(int D, int G) {
+#define TRI_CASE(DD, GG) \
+    if (D == DD && G == GG) return &tri::tri_fused_kernel<DD, GG, 0, true>;
+    TRI_CASE(64, 1) TRI_CASE(64, 2) TRI_CASE(64, 4) TRI_CASE(64, 8)
+    TRI_CASE(128, 1) TRI_CASE(128, 2) TRI_CASE(128, 4) TRI_CASE(128, 8)
+#undef TRI_CASE
+    return nullptr;
+}
+
+using MxImageFn = void (*)(const tri::MxArgs);
+using MxScoreFn = void (*)(const CUtensorMap, const tri::MxArgs);
+
+bool pick_mx(int D, int G, int layout, MxImageFn *img, MxScoreFn *score) {
+#define TRI_MX_CASE(DD, GG, LL)                                  \
+    if (D == DD && G == GG && layout == LL) {                    \
+        *img = &tri::tri_mx_image_kernel<DD, GG, LL>;            \
+        *score = &tri::tri_mx_score_kernel<DD, GG, LL>;          \
+        return true;                                             \
+    }
+    TRI_MX_CASE(64, 1, 0) TRI_MX_CASE(64, 2, 0) TRI_MX_CASE(64, 4, 0) TRI_MX_CASE(64, 8, 0)
+    TRI_MX_CASE(64, 1, 1) TRI_MX_CASE(64, 2, 1) TRI_MX_CASE(64, 4, 1) TRI_MX_CASE(64, 8, 1)
+    TRI_MX_CASE(128, 1, 0) TRI_MX_CASE(128, 2, 0) TRI_MX_CASE(128, 4, 0) TRI_MX_CASE(128, 8, 0)
+    TRI_MX_CASE(128, 1, 1) TRI_MX_CASE(128, 2, 1) TRI_MX_CASE(128, 4, 1) TRI_MX_CASE(128, 8, 1)
+#undef TRI_MX_CASE
+    return false;
 }
 
 // Device memory check: a pointer the runtime does not know as device or managed memory
@@ -266,8 +317,9 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
     return TRI_OK;
 }
 
-tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
-               int mode, void *stream) {
+// Host checks of a scoring call (tri_prune / tri_score); on success *cap_out is the unit capacity.
+tri_status check_call(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
+                      int mode, long long *cap_out) {
     if (!c || !kv || !t) return TRI_EINVAL;
     if (!c->loaded) return TRI_ESTATE;
     if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
@@ -301,9 +353,29 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
 
     const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
     if (n_units * tri::kMaxCluster > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+    *cap_out = cap_u;
+    return TRI_OK;
+}
 
-    KernelFn fn = pick_kernel(c->D, c->G, c->layout);
-    if (!fn) return TRI_EUNSUPPORTED;
+tri_status ensure_seq_bad(tri_ctx *c, int batch) {
+    if (batch <= c->seq_bad_cap) return TRI_OK;
+    cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
+    c->d_seq_bad = nullptr;
+    c->seq_bad_cap = 0;
+    if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ENOMEM;
+    if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ECUDA;
+    c->seq_bad_cap = batch;
+    return TRI_OK;
+}
+
+// One launch of the fused kernel `fn` over the units of kv. pre / unit_fail: precomputed
+// scores (the PRE variant) or null; lens_out: where the last CTA publishes the new lengths
+// (null: not in this launch); seq_bad: refusal flags (null: none kept).
+tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw,
+                        float *zmax, int mode, long long cap_u, const float *pre, const int32_t *unit_fail,
+                        long long unit_base, int32_t *lens_out, int32_t *seq_bad, void *stream) {
+    const bool paged = kv->block_table != nullptr;
+    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
     ce = prepare_kernel(fn, c->max_smem_optin);
@@ -323,23 +395,13 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
         c->scratch_bytes = need;
     }
 
-    const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
-    if (finalize && kv->batch > c->seq_bad_cap) {
-        cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
-        c->d_seq_bad = nullptr;
-        c->seq_bad_cap = 0;
-        if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ENOMEM;
-        if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ECUDA;
-        c->seq_bad_cap = kv->batch;
-    }
-
     tri::Args a;
     std::memset(&a, 0, sizeof a);
     a.K = static_cast<uint16_t *>(kv->K);
     a.V = static_cast<uint16_t *>(kv->V);
     a.pos = kv->pos;
     a.lens = kv->lens;
-    a.lens_out = finalize ? kv->lens_out : nullptr;
+    a.lens_out = mode == tri::kModePrune ? lens_out : nullptr;
     a.block_table = kv->block_table;
     a.t = t;
     a.batch = kv->batch;
@@ -366,7 +428,10 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     a.slot_floats = slot_floats;
     a.status = c->d_status;
     a.counter = c->d_counter;
-    a.seq_bad = finalize ? c->d_seq_bad : nullptr;
+    a.seq_bad = mode == tri::kModePrune ? seq_bad : nullptr;
+    a.pre = pre;
+    a.unit_fail = unit_fail;
+    a.unit_base = unit_base;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
@@ -384,6 +449,204 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     ce = cudaLaunchKernelEx(&cfg, fn, a);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx");
     return TRI_OK;
+}
+
+// Grow a scratch buffer of the context (cudaFree synchronises the device, so no call still
+// uses the old one).
+template <class T>
+tri_status grow(tri_ctx *c, T **p, size_t *cap, size_t need, const char *what) {
+    if (need <= *cap) return TRI_OK;
+    cudaFree(*p);
+    *p = nullptr;
+    *cap = 0;
+    void *q = nullptr;
+    const cudaError_t ce = cudaMalloc(&q, need);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, what, TRI_ENOMEM);
+    *p = static_cast<T *>(q);
+    *cap = need;
+    return TRI_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        else
+            cudaGetLastError();
+    });
+    return fn;
+}
+
+// Scores held for at most this many bytes at a time; longer calls run in chunks of layers.
+constexpr size_t kMaxPreBytes = size_t(1) << 30;
+
+// The max-over-offsets mode: per chunk of layers, the tensor-core scoring kernel writes every
+// unit's scores, then the fused kernel's PRE variant z-scores, selects and compacts.
+tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
+                   int mode, long long cap_u, void *stream) {
+    const int D = c->D, G = c->G, F = D / 2, Hkv = c->Hkv, Hq = Hkv * G;
+    if (G * c->n_off > 256) {
+        std::snprintf(c->last_error, sizeof c->last_error,
+                      "max over offsets: group * n_offsets = %d exceeds the 256 columns of one MMA", G * c->n_off);
+        return TRI_EUNSUPPORTED;
+    }
+    MxImageFn img_fn = nullptr;
+    MxScoreFn score_fn = nullptr;
+    if (!pick_mx(D, G, c->layout, &img_fn, &score_fn)) return TRI_EUNSUPPORTED;
+    KernelFn fused = pick_pre_kernel(D, G);
+    if (!fused) return TRI_EUNSUPPORTED;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
+    if (!encode) {
+        std::snprintf(c->last_error, sizeof c->last_error, "cuTensorMapEncodeTiled is not available");
+        return TRI_ECUDA;
+    }
+    const bool paged = kv->block_table != nullptr;
+    const int ncol = tri::mx_ncol(G, c->n_off);
+    const int acc_cols = tri::mx_acc_cols(ncol);
+    const unsigned img_bytes = tri::mx_image_bytes(D, G, ncol);
+    int piece_rows = 64;
+    if (paged) {
+        piece_rows = kv->page_size % 64 == 0 ? 64 : kv->page_size % 32 == 0 ? 32 : 16;
+    }
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+    cudaFuncAttributes fa;
+    ce = cudaFuncGetAttributes(&fa, score_fn);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncGetAttributes(score)");
+    const size_t smem_budget = (size_t)c->max_smem_optin - fa.sharedSizeBytes;
+    int nst = tri::kMxMaxStages;
+    while (nst >= 2 && tri::mx_layout(D, G, ncol, nst).total > smem_budget) --nst;
+    if (nst < 2) return TRI_EUNSUPPORTED;
+    // at least 120 KB, so that one CTA runs per SM and its TMEM allocation never waits
+    const size_t smem = std::max<size_t>(tri::mx_layout(D, G, ncol, nst).total, 120 * 1024);
+    ce = cudaFuncSetAttribute(score_fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute(score)");
+
+    // layers per chunk: the scores of one chunk stay under kMaxPreBytes
+    const long long units_per_layer = (long long)kv->batch * Hkv;
+    const size_t pre_per_layer = (size_t)units_per_layer * cap_u * G * sizeof(float);
+    const int chunk = (int)std::max<size_t>(1, std::min<size_t>((size_t)kv->n_layers, kMaxPreBytes / pre_per_layer));
+    const long long layer_rows = paged ? (long long)kv->n_pages * Hkv * kv->page_size : units_per_layer * cap_u;
+    if (layer_rows * chunk >= (1LL << 31)) return TRI_EUNSUPPORTED;  // TMA row coordinates are int32
+
+    tri_status st;
+    if ((st = grow(c, &c->d_pre, &c->pre_bytes, pre_per_layer * chunk, "cudaMalloc(scores)")) != TRI_OK) return st;
+    if ((st = grow(c, &c->d_image, &c->image_bytes, (size_t)units_per_layer * chunk * img_bytes,
+                   "cudaMalloc(coefficients)")) != TRI_OK)
+        return st;
+    if ((st = grow(c, &c->d_phase, &c->phase_bytes, (size_t)kv->batch * c->n_off * F * sizeof(double2),
+                   "cudaMalloc(phases)")) != TRI_OK)
+        return st;
+    if ((st = grow(c, &c->d_tile_prefix, &c->tile_prefix_bytes, (size_t)(kv->batch + 1) * sizeof(int32_t),
+                   "cudaMalloc(tile prefix)")) != TRI_OK)
+        return st;
+    if ((st = grow(c, &c->d_unit_fail, &c->unit_fail_bytes, (size_t)units_per_layer * chunk * sizeof(int32_t),
+                   "cudaMalloc(unit flags)")) != TRI_OK)
+        return st;
+    const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
+    if (finalize && (st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+
+    tri::MxArgs m;
+    std::memset(&m, 0, sizeof m);
+    m.lens = kv->lens;
+    m.block_table = kv->block_table;
+    m.t = t;
+    m.batch = kv->batch;
+    m.n_kv = Hkv;
+    m.cap_u = (int)cap_u;
+    m.paged = paged ? 1 : 0;
+    m.page_size = paged ? kv->page_size : 0;
+    m.max_pages = paged ? kv->max_pages : 0;
+    m.n_pages = paged ? kv->n_pages : 0;
+    m.min_len = mode == tri::kModePrune ? budget : 0;
+    m.n_off = c->n_off;
+    m.ncol = ncol;
+    m.acc_cols = acc_cols;
+    m.nst = nst;
+    m.piece_rows = piece_rows;
+    m.qbar = c->d_qbar;
+    m.omega = c->d_omega;
+    m.offsets = c->d_offsets;
+    m.w = c->d_w;
+    m.phase = c->d_phase;
+    m.image = c->d_image;
+    m.tile_prefix = c->d_tile_prefix;
+    m.pre = c->d_pre;
+    m.unit_fail = c->d_unit_fail;
+    m.status = c->d_status;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    tri::tri_mx_prefix_kernel<<<1, 32, 0, cs>>>(m);
+    const long long n_ph = (long long)kv->batch * c->n_off * F;
+    tri::tri_mx_phase_kernel<<<(unsigned)((n_ph + 255) / 256), 256, 0, cs>>>(m, F);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(prefix, phase)");
+
+    for (int lr0 = 0; lr0 < kv->n_layers; lr0 += chunk) {
+        const int nl = std::min(chunk, kv->n_layers - lr0);
+        const long long row0 = (long long)lr0 * layer_rows;
+        tri_kv sub = *kv;
+        sub.layer_begin = kv->layer_begin + lr0;
+        sub.n_layers = nl;
+        sub.K = static_cast<uint16_t *>(kv->K) + row0 * D;
+        if (kv->V) sub.V = static_cast<uint16_t *>(kv->V) + row0 * D;
+        if (kv->pos) sub.pos = kv->pos + row0;
+        float *raw_c = raw ? raw + (long long)lr0 * kv->batch * Hq * cap_u : nullptr;
+        float *zmax_c = zmax ? zmax + (long long)lr0 * units_per_layer * cap_u : nullptr;
+
+        CUtensorMap tmap;
+        const cuuint64_t gdim[2] = {(cuuint64_t)D, (cuuint64_t)(layer_rows * nl)};
+        const cuuint64_t gstride[1] = {(cuuint64_t)D * 2};
+        const cuuint32_t box[2] = {64u, (cuuint32_t)piece_rows};
+        const cuuint32_t estride[2] = {1u, 1u};
+        const CUresult cr = encode(&tmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, sub.K, gdim, gstride, box, estride,
+                                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (cr != CUDA_SUCCESS) {
+            std::snprintf(c->last_error, sizeof c->last_error, "cuTensorMapEncodeTiled failed (%d)", (int)cr);
+            return TRI_ECUDA;
+        }
+        m.layer_begin = sub.layer_begin;
+        m.n_layers = nl;
+        m.unit_base = (long long)lr0 * units_per_layer;
+        const long long nu = (long long)nl * units_per_layer;
+        img_fn<<<(unsigned)nu, 256, 0, cs>>>(m);
+        ce = cudaMemsetAsync(c->d_unit_fail, 0, (size_t)nu * sizeof(int32_t), cs);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaMemsetAsync(unit flags)");
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof cfg);
+        cfg.gridDim = dim3((unsigned)c->sm_count);
+        cfg.blockDim = dim3((unsigned)tri::kMxThreads);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = cs;
+        ce = cudaLaunchKernelEx(&cfg, score_fn, tmap, m);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx(score)");
+        const bool last = lr0 + nl == kv->n_layers;
+        st = launch_fused(c, fused, &sub, t, budget, raw_c, zmax_c, mode, cap_u, c->d_pre, c->d_unit_fail,
+                          m.unit_base, (finalize && last) ? kv->lens_out : nullptr,
+                          finalize ? c->d_seq_bad : nullptr, stream);
+        if (st != TRI_OK) return st;
+    }
+    return TRI_OK;
+}
+
+tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
+               int mode, void *stream) {
+    long long cap_u = 0;
+    tri_status st = check_call(c, kv, t, budget, raw, zmax, mode, &cap_u);
+    if (st != TRI_OK) return st;
+    if (c->combine == TRI_OFFSETS_MAX) return run_max(c, kv, t, budget, raw, zmax, mode, cap_u, stream);
+    KernelFn fn = pick_kernel(c->D, c->G, c->layout);
+    if (!fn) return TRI_EUNSUPPORTED;
+    const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
+    if (finalize && (st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+    return launch_fused(c, fn, kv, t, budget, raw, zmax, mode, cap_u, nullptr, nullptr, 0,
+                        finalize ? kv->lens_out : nullptr, finalize ? c->d_seq_bad : nullptr, stream);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -434,6 +697,11 @@ tri_status noalloc_symbols(tri_ctx *c, NoAllocSymbols *out) {
 tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
     if (!c || !kv || !t) return TRI_EINVAL;
     if (!c->loaded) return TRI_ESTATE;
+    if (c->combine != TRI_OFFSETS_MEAN) {
+        std::snprintf(c->last_error, sizeof c->last_error,
+                      "tri_prune_noalloc: the max-over-offsets mode needs scratch that only tri_prune allocates");
+        return TRI_EUNSUPPORTED;
+    }
     if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
         return TRI_EINVAL;
     const bool paged = kv->block_table != nullptr;
@@ -613,6 +881,11 @@ tri_status tri_destroy(tri_ctx *c) {
     cudaFree(c->d_counter);
     cudaFree(c->d_seq_bad);
     cudaFree(c->d_scratch);
+    cudaFree(c->d_pre);
+    cudaFree(c->d_image);
+    cudaFree(c->d_phase);
+    cudaFree(c->d_tile_prefix);
+    cudaFree(c->d_unit_fail);
     delete c;
     return TRI_OK;
 }
@@ -646,7 +919,7 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
         Are[f] = sr / n_offsets;
         Aim[f] = si / n_offsets;
     }
-    std::vector<double2> Qc(nb);
+    std::vector<double2> Qc(nb), qbar(nb);
     std::vector<float> w(nb);
     for (size_t lh = 0; lh < (size_t)n_layers * Hq; ++lh) {
         const float *q = q_mean + lh * D;
@@ -655,6 +928,7 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
             const int dim = layout == TRI_ROPE_HALF ? f + F : 2 * f + 1;
             const double qr = q[dre], qi = q[dim];
             Qc[lh * F + f] = make_double2(qr * Are[f] - qi * Aim[f], qr * Aim[f] + qi * Are[f]);
+            qbar[lh * F + f] = make_double2(qr, qi);
             w[lh * F + f] = (float)((1.0 - (double)R[lh * F + f]) * (double)q_norm_mean[lh * F + f]);
         }
     }
@@ -662,16 +936,21 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
     free_stats(c);
     if (cudaMalloc(&c->d_omega, sizeof(double) * F) != cudaSuccess ||
         cudaMalloc(&c->d_Qc, sizeof(double2) * nb) != cudaSuccess ||
-        cudaMalloc(&c->d_w, sizeof(float) * nb) != cudaSuccess) {
+        cudaMalloc(&c->d_w, sizeof(float) * nb) != cudaSuccess ||
+        cudaMalloc(&c->d_qbar, sizeof(double2) * nb) != cudaSuccess ||
+        cudaMalloc(&c->d_offsets, sizeof(int64_t) * n_offsets) != cudaSuccess) {
         free_stats(c);
         return TRI_ENOMEM;
     }
     if (cudaMemcpy(c->d_omega, omega.data(), sizeof(double) * F, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->d_Qc, Qc.data(), sizeof(double2) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(c->d_w, w.data(), sizeof(float) * nb, cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaMemcpy(c->d_w, w.data(), sizeof(float) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->d_qbar, qbar.data(), sizeof(double2) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemcpy(c->d_offsets, offsets, sizeof(int64_t) * n_offsets, cudaMemcpyHostToDevice) != cudaSuccess) {
         free_stats(c);
         return TRI_ECUDA;
     }
+    c->n_off = n_offsets;
     c->L = n_layers;
     c->Hkv = n_kv_heads;
     c->G = group;
@@ -791,6 +1070,13 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
                                                                                        c->d_seq_bad, kv->batch);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append lengths");
+    return TRI_OK;
+}
+
+tri_status tri_set_offset_combine(tri_ctx *c, int combine) {
+    if (!c) return TRI_EINVAL;
+    if (combine != TRI_OFFSETS_MEAN && combine != TRI_OFFSETS_MAX) return TRI_EINVAL;
+    c->combine = combine;
     return TRI_OK;
 }
 

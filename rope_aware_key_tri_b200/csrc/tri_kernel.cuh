@@ -94,6 +94,9 @@ struct Args {
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
     int32_t *seq_bad;            // [batch] sequences the device refused this call
+    const float *pre;            // precomputed scores [n_units][cap_u][G] (max-over-offsets mode)
+    const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing
+    long long unit_base;         // added to the unit index in device status reports
 };
 
 // Per-CTA values other CTAs of the cluster read through distributed shared memory.
@@ -415,7 +418,9 @@ __host__ __device__ constexpr int pair_dim(int p, int e) {
 // ---------------------------------------------------------------------------------
 // The fused kernel. Grid: n_clusters * cs CTAs (clusters of cs), persistent over units.
 // ---------------------------------------------------------------------------------
-template <int D, int G, int LAYOUT>
+// PRE: the scores come precomputed (one [cap_u][G] row block per unit) instead of being
+// computed here; the z-score, select and compaction are the same.
+template <int D, int G, int LAYOUT, bool PRE = false>
 __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(const Args a) {
     constexpr int kWarps = cta_warps(G);
     constexpr int kThreads = kWarps * 32;
@@ -516,10 +521,13 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             if (__syncthreads_or(mine)) bad = kDevBadPage;
         }
         if (bad && crank == 0 && tid == 0) {
-            record_status(a.status, bad, unit);
+            record_status(a.status, bad, a.unit_base + unit);
             if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
-        const bool work = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
+        bool missing = false;  // the scoring kernel gave up on this unit (it recorded why)
+        if constexpr (PRE) missing = !bad && __ldg(a.unit_fail + unit) != 0;
+        if (missing && crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
+        const bool work = !bad && !missing && N > 0 && (a.mode == kModeScore || N > a.budget);
         if (!work) continue;  // uniform over the cluster: no cluster barrier is skipped unevenly
 
         const int kpc = ((N + cs - 1) / cs + 31) / 32 * 32;
@@ -528,6 +536,14 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
         const int nst = (n_local + kStageRows - 1) / kStageRows;
         const int my_stages = warp < nst ? (nst - warp + kWarps - 1) / kWarps : 0;
 
+        float *sc_local = sc + (long long)begin * G;
+        const float *sc_read = sc_local;  // where the z pass reads this CTA's scores
+        double m_s = 0.0, m_q = 0.0;
+        float m_lo = __int_as_float(0x7f800000), m_hi = -__int_as_float(0x7f800000);
+        int fail = 0;
+        if constexpr (PRE) {
+            sc_read = a.pre + ((long long)unit * a.cap_u + begin) * G;
+        } else {
         // ---- start streaming this CTA's keys (TMA bulk copies, per-warp buffers) -----
         auto issue = [&](int st) {
             const int slot = wr_slot;
@@ -593,14 +609,10 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
                 cw[i][p] = make_float2(coef_w[hq * F + b0], coef_w[hq * F + b0 + 1]);
             }
         }
-        float *sc_local = sc + (long long)begin * G;
 
         // ---- score loop ----------------------------------------------------------------
         // writer lanes also gather their head's moments (fp64 sum and sum of squares, fp32
         // min and max) so that the scores are read back only once, for the z-score
-        double m_s = 0.0, m_q = 0.0;
-        float m_lo = __int_as_float(0x7f800000), m_hi = -__int_as_float(0x7f800000);
-        int fail = 0;
         for (int k = 0; k < my_stages; ++k) {
             const int st = warp + k * kWarps;
             const int slot = rd_slot;
@@ -692,9 +704,10 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
                 if (++wr_slot == nslot) wr_slot = 0;
             }
         }
+        }  // !PRE
         if (__syncthreads_or(fail)) {
             if (tid == 0) {
-                record_status(a.status, kDevTimeout, unit);
+                record_status(a.status, kDevTimeout, a.unit_base + unit);
                 if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
             }
             fail = 1;
@@ -705,6 +718,49 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
         // a fixed order, then the warps in order, then the cluster's CTAs in rank order, so
         // that every CTA obtains bit-identical mu and sigma.
         {
+            if constexpr (PRE) {
+                // every thread folds all G heads of its keys, then the warp folds its lanes
+                double ps[G], pq[G];
+                float plo[G], phi[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    ps[h] = 0.0;
+                    pq[h] = 0.0;
+                    plo[h] = __int_as_float(0x7f800000);
+                    phi[h] = -__int_as_float(0x7f800000);
+                }
+                for (int i = tid; i < n_local; i += kThreads) {
+                    float sv[G];
+                    load_scores<G>(sc_read + (long long)i * G, sv);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const double dv = (double)sv[h];
+                        ps[h] += dv;
+                        pq[h] = fma(dv, dv, pq[h]);
+                        plo[h] = fminf(plo[h], sv[h]);
+                        phi[h] = fmaxf(phi[h], sv[h]);
+                    }
+                }
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        ps[h] += __shfl_xor_sync(FULL, ps[h], o);
+                        pq[h] += __shfl_xor_sync(FULL, pq[h], o);
+                        plo[h] = fminf(plo[h], __shfl_xor_sync(FULL, plo[h], o));
+                        phi[h] = fmaxf(phi[h], __shfl_xor_sync(FULL, phi[h], o));
+                    }
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        w_s[warp][h] = ps[h];
+                        w_q[warp][h] = pq[h];
+                        w_lo[warp][h] = plo[h];
+                        w_hi[warp][h] = phi[h];
+                    }
+                }
+            } else {
 #pragma unroll
             for (int o = LPK; o < 32; o <<= 1) {
                 m_s += __shfl_xor_sync(FULL, m_s, o);
@@ -717,6 +773,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
                 w_q[warp][hx] = m_q;
                 w_lo[warp][hx] = m_lo;
                 w_hi[warp][hx] = m_hi;
+            }
             }
             __syncthreads();
             if (tid < G) {
@@ -806,7 +863,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
 #pragma unroll
                 for (int k = 0; k < ZB; ++k) {
                     const int i = base + k * kThreads;
-                    if (i < n_local) load_scores<G>(sc_local + i * G, sv[k]);
+                    if (i < n_local) load_scores<G>(sc_read + (long long)i * G, sv[k]);
                 }
 #pragma unroll
                 for (int k = 0; k < ZB; ++k) {
@@ -826,7 +883,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             if (raw_row) {
                 for (int i = tid; i < n_local; i += kThreads) {
                     float sv[G];
-                    load_scores<G>(sc_local + i * G, sv);
+                    load_scores<G>(sc_read + (long long)i * G, sv);
 #pragma unroll
                     for (int h = 0; h < G; ++h) raw_row[(long long)h * a.cap_u + i] = sv[h];
                 }
@@ -962,7 +1019,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             // unit is left untouched rather than copied from a wrong index
             const bool count_ok = total == M;
             if (!count_ok && crank == 0 && tid == 0) {
-                record_status(a.status, kDevInternal, unit);
+                record_status(a.status, kDevInternal, a.unit_base + unit);
                 if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
             }
 

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libtri_b200.so")
 
 TRI_OK, TRI_EINVAL, TRI_ENOMEM, TRI_ECUDA, TRI_ESTATE, TRI_EDEVICE, TRI_EUNSUPPORTED = range(7)
 TRI_ROPE_HALF, TRI_ROPE_INTERLEAVED = 0, 1
+TRI_OFFSETS_MEAN, TRI_OFFSETS_MAX = 0, 1
 TRI_DEV_NONE, TRI_DEV_LEN_GT_CAP, TRI_DEV_BAD_PAGE, TRI_DEV_TIMEOUT, TRI_DEV_INTERNAL = range(5)
 
 
@@ -67,12 +68,14 @@ def _load():
     L.tri_append.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
     L.tri_set_tuning.argtypes = [P, ctypes.c_int, ctypes.c_int]
+    L.tri_set_offset_combine.argtypes = [P, ctypes.c_int]
     L.tri_last_error.argtypes = [P]
     L.tri_last_error.restype = ctypes.c_char_p
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
     for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
-               "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_set_tuning", "tri_version"):
+               "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_set_tuning", "tri_set_offset_combine",
+               "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
     return L
 
@@ -159,6 +162,10 @@ def tri_set_tuning(ctx, cluster_size: int = 0, buffers_per_warp: int = 0) -> int
     return _lib.tri_set_tuning(ctx, int(cluster_size), int(buffers_per_warp))
 
 
+def tri_set_offset_combine(ctx, combine: int) -> int:
+    return _lib.tri_set_offset_combine(ctx, int(combine))
+
+
 # ---- torch-facing wrapper ----------------------------------------------------------------
 
 def _ptr(x: Optional[torch.Tensor]) -> Optional[int]:
@@ -224,6 +231,13 @@ class TriContext:
                                 q_mean, q_norm_mean, R, offsets)
         if st != TRI_OK:
             raise TriError(st, "tri_calibrate_load")
+
+    def set_offset_combine(self, combine):
+        """"mean" (the default) or "max" over the future offsets (or the TRI_OFFSETS_* value)."""
+        code = {"mean": TRI_OFFSETS_MEAN, "max": TRI_OFFSETS_MAX}.get(combine, combine)
+        st = tri_set_offset_combine(self.handle, code)
+        if st != TRI_OK:
+            raise TriError(st, "tri_set_offset_combine")
 
     def set_tuning(self, cluster_size=0, buffers_per_warp=0):
         st = tri_set_tuning(self.handle, cluster_size, buffers_per_warp)

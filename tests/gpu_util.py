@@ -19,13 +19,15 @@ SCORE_RTOL = 1e-4
 Z_TIE = 1e-4
 
 
-def context_for(cache, cluster_size=0, buffers=0):
+def context_for(cache, cluster_size=0, buffers=0, combine="mean"):
     s = cache.spec
     ctx = tri.TriContext(0)
     ctx.calibrate_load(s.n_layers, s.n_kv_heads, s.group, s.head_dim, s.rope_base, s.layout,
                        cache.q_mean, cache.q_norm_mean, cache.R, cache.offsets)
     if cluster_size or buffers:
         ctx.set_tuning(cluster_size, buffers)
+    if combine != "mean":
+        ctx.set_offset_combine(combine)
     return ctx
 
 
@@ -52,13 +54,13 @@ def gpu_prune(ctx, cache, budget=None, lens_out="inplace"):
     return ctx.get_error()
 
 
-def oracle_unit(cache, u, B, rows=None):
+def oracle_unit(cache, u, B, rows=None, combine="mean"):
     s = cache.spec
     k, v, p = rows if rows is not None else cache.unit_rows(u)
     qm, qn, R = cache.unit_stats(u)
     _, b, _ = cache.unit_index(u)
     return oracle.prune_unit(k, v, p, int(cache.t_host[b]), qm, qn, R, cache.offsets, s.rope_base, B,
-                             s.layout)
+                             s.layout, combine=combine)
 
 
 def check_scores(raw_u, zmax_u, orc, label=""):

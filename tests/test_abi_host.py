@@ -27,7 +27,8 @@ def lib():
 def test_header_declares_the_boundary():
     names = _declared()
     for n in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_score",
-              "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_status_str"):
+              "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_status_str",
+              "tri_set_offset_combine"):
         assert n in names
 
 
@@ -53,6 +54,7 @@ def test_host_validation_without_device(lib):
     assert lib.tri_score(None, ctypes.byref(kv), None, None, None, None) == tri.TRI_EINVAL
     assert lib.tri_destroy(None) == tri.TRI_OK
     assert lib.tri_set_tuning(None, 0, 0) == tri.TRI_EINVAL
+    assert lib.tri_set_offset_combine(None, tri.TRI_OFFSETS_MAX) == tri.TRI_EINVAL
     assert tri.tri_calibrate_estimate(None, None, 1, 1, 1, 128, 0, None, None, None, None) == tri.TRI_EINVAL
     assert lib.tri_append(None, ctypes.byref(kv), None, None, None, None) == tri.TRI_EINVAL
     assert lib.tri_calibrate_load(None, 1, 1, 1, 64, ctypes.c_double(1e4), 0, None, None, None, None, 1) \

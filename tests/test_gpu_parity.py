@@ -36,10 +36,10 @@ def _written_mask_dense(cache, M_of_seq):
     return m
 
 
-def full_parity(cache, budget=None, cluster_size=0, check_scores=True, label=""):
+def full_parity(cache, budget=None, cluster_size=0, check_scores=True, label="", combine="mean"):
     s = cache.spec
     B = s.budget if budget is None else budget
-    ctx = gu.context_for(cache, cluster_size)
+    ctx = gu.context_for(cache, cluster_size, combine=combine)
     if check_scores:
         raw, zmx = gu.gpu_score(ctx, cache)
     rows_in = [cache.unit_rows(u) for u in range(cache.n_units)]
@@ -53,7 +53,7 @@ def full_parity(cache, budget=None, cluster_size=0, check_scores=True, label="")
     for u in range(cache.n_units):
         l, b, g = cache.unit_index(u)
         lab = f"{label} unit {u} (l={l}, s={b}, g={g}, N={lens_before[b]})"
-        orc = gu.oracle_unit(cache, u, B, rows=rows_in[u])
+        orc = gu.oracle_unit(cache, u, B, rows=rows_in[u], combine=combine)
         if check_scores:
             gu.check_scores(raw[l, b, g * s.group:(g + 1) * s.group], zmx[l, b, g], orc, lab)
         out = cache.unit_rows(u)
