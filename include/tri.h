@@ -284,6 +284,11 @@ TRI_API tri_status tri_set_tuning(tri_ctx *ctx, int cluster_size, int buffers_pe
  */
 TRI_API tri_status tri_set_offset_combine(tri_ctx *ctx, int combine);
 
+/* Tracing: tri_prune, tri_prune_noalloc, tri_score, tri_calibrate_estimate and tri_append each
+ * mark their host-side span (argument checks and launches) with an NVTX range in the domain
+ * "tri"; the max-over-offsets mode adds one range per chunk of layers. A timeline profiler shows
+ * them; without one they cost a few nanoseconds. */
+
 /* Text of the last host-side failure on this context (the CUDA error and the call that
  * returned it), or an empty string. Valid until the next call on the context. */
 TRI_API const char *tri_last_error(tri_ctx *ctx);

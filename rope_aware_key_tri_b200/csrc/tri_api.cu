@@ -10,6 +10,7 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -74,6 +75,29 @@ struct tri_ctx {
 };
 
 namespace {
+
+// NVTX ranges (domain "tri") around every entry point that launches work, so that a timeline
+// profiler shows each call and, in the max-over-offsets mode, each chunk of layers. Without a
+// profiler attached a range costs a couple of branches.
+nvtxDomainHandle_t nvtx_domain() {
+    static nvtxDomainHandle_t d = nvtxDomainCreateA("tri");
+    return d;
+}
+
+struct NvtxRange {
+    explicit NvtxRange(const char *name) {
+        nvtxEventAttributes_t e;
+        std::memset(&e, 0, sizeof e);
+        e.version = NVTX_VERSION;
+        e.size = NVTX_EVENT_ATTRIB_STRUCT_SIZE;
+        e.messageType = NVTX_MESSAGE_TYPE_ASCII;
+        e.message.ascii = name;
+        nvtxDomainRangePushEx(nvtx_domain(), &e);
+    }
+    ~NvtxRange() { nvtxDomainRangePop(nvtx_domain()); }
+    NvtxRange(const NvtxRange &) = delete;
+    NvtxRange &operator=(const NvtxRange &) = delete;
+};
 
 using KernelFn = void (*)(const tri::Args);
 
@@ -588,6 +612,7 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
     if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(prefix, phase)");
 
     for (int lr0 = 0; lr0 < kv->n_layers; lr0 += chunk) {
+        NvtxRange chunk_range("tri max-over-offsets: chunk of layers");
         const int nl = std::min(chunk, kv->n_layers - lr0);
         const long long row0 = (long long)lr0 * layer_rows;
         tri_kv sub = *kv;
@@ -961,20 +986,24 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
 }
 
 tri_status tri_prune(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
+    NvtxRange r("tri_prune");
     return run(c, kv, t, budget, nullptr, nullptr, tri::kModePrune, stream);
 }
 
 tri_status tri_prune_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, void *stream) {
+    NvtxRange r("tri_prune_noalloc");
     return run_noalloc(c, kv, t, budget, stream);
 }
 
 tri_status tri_score(tri_ctx *c, const tri_kv *kv, const int32_t *t, float *raw, float *zmax, void *stream) {
+    NvtxRange r("tri_score");
     return run(c, kv, t, 0, raw, zmax, tri::kModeScore, stream);
 }
 
 tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T, int n_q_heads, int head_dim,
                                   tri_rope_layout layout, float *q_mean, float *q_norm_mean, float *R,
                                   void *stream) {
+    NvtxRange r("tri_calibrate_estimate");
     if (!c || !Q || !q_mean || !q_norm_mean || !R) return TRI_EINVAL;
     if (n_layers < 1 || T < 1 || n_q_heads < 1) return TRI_EINVAL;
     if (layout != TRI_ROPE_HALF && layout != TRI_ROPE_INTERLEAVED) return TRI_EINVAL;
@@ -1015,6 +1044,7 @@ tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T
 
 tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, const int32_t *pos_new,
                       void *stream) {
+    NvtxRange r("tri_append");
     if (!c || !kv || !K_new || !V_new || !pos_new) return TRI_EINVAL;
     if (!c->loaded) return TRI_ESTATE;
     if (c->D != 64 && c->D != 128) return TRI_EUNSUPPORTED;
