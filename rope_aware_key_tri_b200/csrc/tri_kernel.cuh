@@ -502,12 +502,22 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
     const bool writer = (sub & (LPK / G - 1)) == 0;
     const int Hq = a.n_kv * G;
 
+    // set once a bounded wait of this cluster ran out: the ring's barrier phases can no longer
+    // be trusted, so the cluster refuses its remaining units instead of streaming them
+    bool dead = false;
     for (int unit = cid; unit < a.n_units; unit += n_clusters) {
         const int g = unit % a.n_kv;
         const int s = (unit / a.n_kv) % a.batch;
         const int lr = unit / (a.n_kv * a.batch);
         const int layer = a.layer_begin + lr;
         const int N = __ldg(a.lens + s);
+        if (dead) {  // uniform over the cluster
+            if (crank == 0 && tid == 0) {
+                record_status(a.status, kDevTimeout, a.unit_base + unit);
+                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
+            }
+            continue;
+        }
 
         // ---- validation: every CTA of the cluster reaches the same verdict ----------
         int bad = (N < 0 || N > a.cap_u) ? kDevLenGtCap : 0;
@@ -830,6 +840,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             anyfail_s = f;
         }
         __syncthreads();
+        dead = anyfail_s != 0;
 
         // ---- z-score, max over the group, order key --------------------------------------
         // The order keys live in the (now idle) TMA ring when they fit, else in the scratch

@@ -32,8 +32,9 @@
 // allocation and issues the MMAs, warps 2-5 run the epilogue. Key tiles stream through a
 // ring of NST stages; accumulators are double-buffered in TMEM; the coefficient image is
 // double-buffered in shared memory and reloaded only when the CTA's tile range enters a new
-// unit. Every wait is bounded; a wait that runs out records a device status, marks the unit
-// so that the fused kernel leaves it untouched, and ends the CTA's work.
+// unit. Every wait is bounded; a wait that runs out records a device status, marks every unit
+// of the CTA's tile range so that the fused kernel leaves them untouched, and ends the CTA's
+// work.
 #pragma once
 
 #include <cuda.h>
@@ -349,10 +350,22 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
+    // A wait that ran out ends the CTA's work: every unit its tile range touches is marked, so
+    // that the next kernel leaves all of them untouched (their scores may be incomplete).
     auto fail = [&](int unit) {
         record_status(a.status, kDevTimeout, a.unit_base + unit);
-        atomicExch(a.unit_fail + unit, 1);
         *abort_flag = 1;
+        MxWalk w2;
+        w2.start(a, T0, per_layer);
+        int last = -1;
+        for (int k = 0; k < count; ++k) {
+            const int u = w2.unit(a);
+            if (u != last) {
+                atomicExch(a.unit_fail + u, 1);
+                last = u;
+            }
+            if (k + 1 < count) w2.next(a);
+        }
     };
 
     if (warp == 0) {
