@@ -13,7 +13,7 @@ import torch
 import tri_synth as ts
 import gpu_util as gu
 from rope_aware_key_tri_b200 import tri
-from test_gpu_parity import full_parity
+from test_gpu_parity import _same, _small, _snapshot, full_parity
 
 pytestmark = pytest.mark.gpu
 
@@ -110,3 +110,75 @@ def test_max_noalloc_refused():
                           block_table=cache.block_table)
     assert e.value.status == tri.TRI_EUNSUPPORTED
     ctx.close()
+
+
+def test_max_edge_lengths_and_noop():
+    """N = 0, 1, B, B + 1 and N < B in one batch: only the unit above the budget is scored and
+    pruned; the others keep their rows and lengths."""
+    B = 40
+    spec = ts.CacheSpec(name="mx_edges", head_dim=128, group=4, n_kv_heads=2, n_layers=1, batch=5,
+                        rope_base=1e6, budget=B, offsets=ts.pow2_offsets(16), positions="from_zero",
+                        lens=(0, 1, B, B + 1, 25), cap=64)
+    cache = ts.make_cache(spec, 4).to("cuda")
+    full_parity(cache, label="max edges", combine="max")
+
+
+def test_max_layer_chunks_match_one_call():
+    """Layer by layer (lens_out NULL, lengths updated at the end) equals one call, in max mode."""
+    spec = _small("qwen3_8b_periodic_36l_3200", n_layers=3, batch=2, n_kv_heads=2, lens=(700, 900),
+                  t=(24576, 24576), budget=512)
+    a = ts.make_cache(spec, 8).to("cuda")
+    b = a.clone()
+    ctx = gu.context_for(a, combine="max")
+    ctx.prune(a.K, a.V, a.pos, a.lens, a.t, spec.budget)
+    for l in range(spec.n_layers):
+        ctx.prune(b.K[l:l + 1], b.V[l:l + 1], b.pos[l:l + 1], b.lens, b.t, spec.budget,
+                  lens_out=None, layer_begin=l)
+    assert torch.equal(b.lens.cpu(), torch.tensor([700, 900], dtype=torch.int32))
+    b.lens.clamp_(max=spec.budget)
+    assert _same(a.K, b.K) and _same(a.V, b.V) and _same(a.pos, b.pos)
+    assert torch.equal(a.lens, b.lens)
+    ctx.close()
+
+
+def test_max_device_detected_errors_leave_sequence_untouched():
+    spec = ts.CacheSpec(name="mx_bad", head_dim=128, group=4, n_kv_heads=2, n_layers=1, batch=3,
+                        rope_base=1e6, budget=30, offsets=ts.pow2_offsets(16), positions="from_zero",
+                        lens=(100, 100, 100), cap=128)
+    cache = ts.make_cache(spec, 6).to("cuda")
+    K0, V0, P0 = _snapshot(cache)
+    cache.lens[1] = 129  # above the capacity
+    ctx = gu.context_for(cache, combine="max")
+    ctx.prune(cache.K, cache.V, cache.pos, cache.lens, cache.t, 30)
+    st, code, unit = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == tri.TRI_DEV_LEN_GT_CAP
+    assert cache.unit_index(unit)[1] == 1
+    assert _same(cache.K[:, 1], K0[:, 1]) and _same(cache.pos[:, 1], P0[:, 1])
+    assert cache.lens_host.tolist() == [30, 129, 30]
+    ctx.close()
+
+    # paged: a block-table entry outside the pool (the scoring kernel loads none of it)
+    pspec = _small("qwen3_32b_paged_ragged", n_layers=1, batch=2, lens=(200, 300), budget=64, cap=512)
+    pc = ts.make_cache(pspec, 7).to("cuda")
+    K0, V0, P0 = _snapshot(pc)
+    pc.block_table[0, 1] = pc.n_pages + 5
+    ctx = gu.context_for(pc, combine="max")
+    ctx.prune(pc.K, pc.V, pc.pos, pc.lens, pc.t, 64, block_table=pc.block_table)
+    st, code, unit = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == tri.TRI_DEV_BAD_PAGE
+    assert pc.lens_host.tolist() == [200, 64]
+    for p in range(4):
+        if p == 1:
+            continue
+        pg = int(pc.block_table_host[0, p])
+        assert _same(pc.K[:, pg], K0[:, pg]) and _same(pc.pos[:, pg], P0[:, pg])
+    ctx.close()
+
+
+@pytest.mark.parametrize("page_size", [32, 48])
+def test_max_prune_paged_odd_pages(page_size):
+    """Pages of 32 and 48 slots: the key tiles are loaded in boxes of 32 and 16 rows."""
+    spec = ts.replace(ts.WORKLOADS["qwen3_32b_paged_ragged"], n_layers=1, batch=2, lens=(400, 257),
+                      page_size=page_size, budget=100, cap=480)
+    cache = ts.make_cache(spec, 31).to("cuda")
+    full_parity(cache, label=f"max paged{page_size}", combine="max")
