@@ -20,6 +20,9 @@ from rope_aware_key_tri_b200 import tri
 pytestmark = pytest.mark.gpu
 
 NAMES = ["qwen3_8b_periodic_36l_3200", "qwen3_8b_oneshot_32k_to_3072", "qwen3_32b_paged_ragged"]
+# every workload in the default (mean over offsets) mode, and the benchmark's one-shot prune in
+# the max-over-offsets mode as well
+CASES = [(n, "mean") for n in NAMES] + [("qwen3_8b_oneshot_32k_to_3072", "max")]
 
 
 def _need_bytes(spec):
@@ -61,8 +64,8 @@ def _hash_all(flat, coeff, chunk=1 << 20):
     return torch.cat([_hash_rows(flat[i:i + chunk], coeff) for i in range(0, flat.shape[0], chunk)])
 
 
-@pytest.mark.parametrize("name", NAMES)
-def test_full_size_workload(name):
+@pytest.mark.parametrize("name,combine", CASES, ids=[f"{n}-{c}" for n, c in CASES])
+def test_full_size_workload(name, combine):
     import gc
     gc.collect()
     torch.cuda.empty_cache()
@@ -76,7 +79,7 @@ def test_full_size_workload(name):
     B = s.budget
     U = cache.n_units
     lens = cache.lens_host.astype(np.int64)
-    ctx = gu.context_for(cache)
+    ctx = gu.context_for(cache, combine=combine)
 
     # ---- sampled units: host copies before anything runs --------------------------------
     rng = np.random.default_rng(7)
@@ -113,7 +116,7 @@ def test_full_size_workload(name):
     for u in picks:
         l, b, g = cache.unit_index(u)
         lab = f"{name} unit {u} (l={l}, s={b}, g={g}, N={lens[b]})"
-        orc = gu.oracle_unit(cache, u, B, rows=rows_in[u])
+        orc = gu.oracle_unit(cache, u, B, rows=rows_in[u], combine=combine)
         gu.check_scores(raw_of[l][b, g * s.group:(g + 1) * s.group], zmx[l, b, g].cpu().numpy(), orc, lab)
         out = cache.unit_rows(u)
         kept = gu.kept_from_output(rows_in[u][2], out[2])
