@@ -55,6 +55,8 @@ def _bind(L):
     L.tri_oracle_unit_scores_max.restype = i32
     L.tri_oracle_calibrate.argtypes = [P, i32, i32, i32, i32, i32, P, P, P]
     L.tri_oracle_calibrate.restype = i32
+    L.tri_oracle_decode_attention.argtypes = [i32, i32, i32, P, P, P, P]
+    L.tri_oracle_decode_attention.restype = i32
     return L
 
 
@@ -183,3 +185,21 @@ def calibrate(Q_bits, layout=HALF, L=None):
     if rc != 0:
         raise ValueError("tri_oracle_calibrate: bad arguments")
     return qm, qn, R
+
+
+def decode_attention(q_bits, K_bits, V_bits, L=None):
+    """Scaled dot-product attention of the G query heads over the M kept rows of one unit.
+
+    q_bits uint16 [G][d], K_bits / V_bits uint16 [M][d] (bf16 bits, post-RoPE query and keys).
+    Returns fp64 [G][d].
+    """
+    Lb = L or lib()
+    q_bits = _c(q_bits, np.uint16); K_bits = _c(K_bits, np.uint16); V_bits = _c(V_bits, np.uint16)
+    G, d = q_bits.shape
+    M = K_bits.shape[0]
+    if K_bits.shape != (M, d) or V_bits.shape != (M, d):
+        raise ValueError("K and V must be [M][d] like the query's d")
+    out = np.zeros((G, d), dtype=np.float64)
+    if Lb.tri_oracle_decode_attention(d, G, M, _p(q_bits), _p(K_bits), _p(V_bits), _p(out)) != 0:
+        raise ValueError("tri_oracle_decode_attention: bad arguments")
+    return out

@@ -50,6 +50,11 @@
  * §3.4 offline calibration; [Stage] §TriAttention：把理论变成算法 items 1-2):
  * the complex centre E[q_f], the mean modulus E|q_f|, and the concentration
  * R_f = |E[q_f]| / E|q_f| of [Stage] §破局之道, taken per band.
+ *
+ * The consumer of the pruned cache (tri_oracle_decode_attention) is the standard scaled
+ * dot-product attention of each query head over the unit's kept rows: softmax of
+ * q.k / sqrt(d) over the keys, applied to the values, as the page "TriAttention 深度解析：
+ * MIT韩松团队如何用三角函数让单卡4090跑出百万Token上下文" writes it out in its section 二.
  */
 #include <math.h>
 #include <stdint.h>
@@ -401,5 +406,50 @@ int tri_oracle_calibrate(const uint16_t *Q, int L, int T, int Hq, int d, int lay
             }
         }
     }
+    return 0;
+}
+
+/*
+ * Decode attention over one pruned unit: the consumer of the compacted cache. For every
+ * query head h of the group, the standard scaled dot-product attention that the
+ * "TriAttention 深度解析：MIT韩松团队如何用三角函数让单卡4090跑出百万Token上下文" page writes out
+ * in its section 二 (logits q.k / sqrt(d), softmax over the cached keys, weights applied to
+ * the values), evaluated on the M rows that the prune kept. The query is post-RoPE (rotated
+ * at its own position t) like the stored keys, so each logit already depends on t - p only
+ * and the kept keys' scattered positions need no other treatment.
+ *   q     [G][d] bf16 bits of the post-RoPE queries of the group
+ *   K, V  [M][d] bf16 bits of the kept (post-RoPE) keys and their values
+ *   out   [G][d] fp64 attention outputs
+ * The largest logit is subtracted before the exponentials (the same softmax, written so that
+ * no exponential overflows). Returns 0, or -1 on bad arguments (M < 1 has no softmax).
+ */
+int tri_oracle_decode_attention(int d, int G, int M, const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                                double *out)
+{
+    if (d < 1 || G < 1 || M < 1 || !q || !K || !V || !out) return -1;
+    const double scale = 1.0 / sqrt((double)d);
+    double *logit = (double *)malloc(sizeof(double) * (size_t)M);
+    if (!logit) return -1;
+    for (int h = 0; h < G; ++h) {
+        double top = -INFINITY;
+        for (int j = 0; j < M; ++j) {
+            double dot = 0.0;
+            for (int i = 0; i < d; ++i)
+                dot += bf16_value(q[(size_t)h * d + i]) * bf16_value(K[(size_t)j * d + i]);
+            logit[j] = dot * scale;
+            if (logit[j] > top) top = logit[j];
+        }
+        double denom = 0.0;
+        for (int j = 0; j < M; ++j) {
+            logit[j] = exp(logit[j] - top);
+            denom += logit[j];
+        }
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < M; ++j) acc += logit[j] * bf16_value(V[(size_t)j * d + i]);
+            out[(size_t)h * d + i] = acc / denom;
+        }
+    }
+    free(logit);
     return 0;
 }

@@ -368,8 +368,46 @@ def pin_calibrate_invariants(L, seed=8):
     assert np.array_equal(ch, ci) and np.array_equal(qh, qi) and np.array_equal(Rh, Ri)
 
 
+def pin_attention_special_cases(L, seed=10):
+    """Decode attention over kept rows: one key returns its value row exactly; identical keys
+    weight every row equally (the mean of the values); permuting the kept rows (keys and
+    values together) changes nothing; a zero query also gives the mean of the values."""
+    r = np.random.default_rng(seed)
+    d, G = 64, 2
+    q = _bf16_bits(r.normal(size=(G, d)))
+    K = _bf16_bits(r.normal(size=(9, d)))
+    V = _bf16_bits(r.normal(size=(9, d)))
+    one = oracle.decode_attention(q, K[:1], V[:1], L=L)
+    assert np.array_equal(one, np.broadcast_to(_bf16_value(V[:1]), (G, d)))
+    same = oracle.decode_attention(q, np.repeat(K[:1], 9, axis=0), V, L=L)
+    assert np.abs(same - _bf16_value(V).mean(axis=0)).max() <= 1e-14
+    zero = oracle.decode_attention(np.zeros_like(q), K, V, L=L)
+    assert np.abs(zero - _bf16_value(V).mean(axis=0)).max() <= 1e-14
+    perm = r.permutation(9)
+    a = oracle.decode_attention(q, K, V, L=L)
+    b = oracle.decode_attention(q, K[perm], V[perm], L=L)
+    assert np.abs(a - b).max() <= 1e-14
+
+
+def pin_attention_library(L, seed=11):
+    """Against torch's scaled_dot_product_attention in float64 (an independent implementation
+    of the same definition), for both head sizes and GQA groups of 1 and 4."""
+    import torch
+    r = np.random.default_rng(seed)
+    for d, G, M in ((64, 1, 5), (128, 4, 300)):
+        q = _bf16_bits(r.normal(scale=2.0, size=(G, d)))
+        K = _bf16_bits(r.normal(size=(M, d)))
+        V = _bf16_bits(r.normal(size=(M, d)))
+        got = oracle.decode_attention(q, K, V, L=L)
+        tq = torch.from_numpy(_bf16_value(q))[None, :, None, :]
+        tk = torch.from_numpy(_bf16_value(K))[None, None].expand(1, G, M, d)
+        tv = torch.from_numpy(_bf16_value(V))[None, None].expand(1, G, M, d)
+        want = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv)[0, :, 0, :].numpy()
+        assert np.abs(got - want).max() <= 1e-12 * max(1.0, np.abs(want).max()), (d, G, M)
+
+
 ALL_PINS = [pin_hand_examples, pin_rope_dot_closed_form, pin_positions_cancel,
             pin_t_shift_is_query_rotation, pin_norm_rotation_invariant_and_linear,
             pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction,
             pin_calibrate_hand_example, pin_calibrate_closed_forms, pin_calibrate_invariants,
-            pin_max_over_delta]
+            pin_max_over_delta, pin_attention_special_cases, pin_attention_library]

@@ -40,6 +40,13 @@ MUTANTS = {
                                     "const double mr = sr / (double)(T - 1), mi = si / (double)(T - 1), mm = sm / (double)(T - 1);"),
     "calib_centre_modulus_first": ("                    sr += re;\n                    si += im;",
                                    "                    sr += fabs(re);\n                    si += fabs(im);"),
+    "attn_scale_by_d": ("const double scale = 1.0 / sqrt((double)d);", "const double scale = 1.0 / (double)d;"),
+    "attn_no_normalisation": ("out[(size_t)h * d + i] = acc / denom;", "out[(size_t)h * d + i] = acc;"),
+    "attn_values_from_keys": ("acc += logit[j] * bf16_value(V[(size_t)j * d + i]);",
+                              "acc += logit[j] * bf16_value(K[(size_t)j * d + i]);"),
+    "attn_first_head_only": ("dot += bf16_value(q[(size_t)h * d + i]) * bf16_value(K[(size_t)j * d + i]);",
+                             "dot += bf16_value(q[i]) * bf16_value(K[(size_t)j * d + i]);"),
+    "attn_minus_logit": ("logit[j] = exp(logit[j] - top);", "logit[j] = exp(top - logit[j]);"),
 }
 
 
