@@ -442,7 +442,7 @@ def run_reference(args, rank, world):
     vals = []
     desc = None
     for i in range(args.warmup + args.steps):
-        v, cores, desc = time_oracle(cache, spec, budget_s=per_step_budget, cores=cores)
+        v, cores, desc = time_oracle(cache, spec, budget_s=per_step_budget, cores=cores, combine=args.combine)
         if i >= args.warmup:
             vals.append(v)
     value = statistics.median(vals)
@@ -452,7 +452,7 @@ def run_reference(args, rank, world):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": args.workload, "layers": spec.n_layers, "kv_heads": spec.n_kv_heads,
                    "group": spec.group, "head_dim": spec.head_dim, "batch": spec.batch,
-                   "budget": spec.budget},
+                   "budget": spec.budget, "offsets_combine": args.combine},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"per step: {desc}"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
