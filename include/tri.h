@@ -15,7 +15,8 @@
  *                    + sum_f (1 - R_f) E|q_f| |k_f|
  *           for each of the G query heads h that share KV head g
  *           ([Stage] §TriAttention：把理论变成算法 items 1-2; [10100] §TriAttention方法;
- *            offsets D of [Deep-dive] §3.3),
+ *            offsets D of [Deep-dive] §3.3); tri_set_offset_combine switches the mean over
+ *           delta to the maximum ([Deep-dive] §3.3 and its §4.2 scoring code),
  *   z/max   z-score each head over the unit's keys, max over the G heads
  *           ([10100] §TriAttention方法; [Summary] §方案设计 item 4),
  *   select  keep the B keys with the largest max-z, ties to the lower slot,
