@@ -103,6 +103,13 @@ def pin_hand_examples(L):
                                      ex["offsets"], ex["base"], LAYOUTS[ex["layout"]], L=L)
         want = np.array([_expr(e) for e in ex["expect"]])
         assert np.allclose(s[:, 0], want, rtol=0, atol=1e-12), (ex["name"], s[:, 0], want)
+    for ex in g["scores_max"]:
+        K = _bf16_bits(np.array(ex["K"], dtype=np.float64))
+        assert np.array_equal(_bf16_value(K), np.array(ex["K"])), ex["name"]
+        s, _, _ = oracle.unit_scores(K, ex["pos"], ex["t"], ex["q_mean"], ex["q_norm"], ex["R"],
+                                     ex["offsets"], ex["base"], LAYOUTS[ex["layout"]], L=L, combine="max")
+        want = np.array([_expr(e) for e in ex["expect"]])
+        assert np.allclose(s[:, 0], want, rtol=0, atol=1e-12), (ex["name"], s[:, 0], want)
     for ex in g["zmax"]:
         z, zm = oracle.zmax(np.array(ex["s"]), L=L)
         assert np.allclose(z[0], [_expr(e) for e in ex["expect_z0"]], atol=1e-12), ex["name"]
