@@ -295,6 +295,63 @@ def pin_max_over_delta(L, seed=9):
             assert np.abs(s2 - s_mx).max() <= 1e-9 * np.abs(s_mx).max()
 
 
+def pin_prune_batch_matches_units(L, seed=12):
+    """The batch driver (threads over units, one flat buffer per argument) gives, unit by
+    unit, what the single-unit pass gives on that unit's own slice: same kept slots, count and
+    max-z, for ragged lengths (0, 1, B, B + 1 and random), groups 1/4/8, both head sizes and
+    rotary layouts, and both ways of combining the offsets. A wrong per-unit offset into any
+    of the flat inputs or outputs reads or writes another unit's data and fails here."""
+    rng = np.random.default_rng(seed)
+    cases = ((64, 1, oracle.HALF, "mean"), (64, 4, oracle.INTERLEAVED, "max"),
+             (128, 8, oracle.HALF, "max"), (128, 4, oracle.INTERLEAVED, "mean"),
+             (128, 2, oracle.HALF, "mean"))
+    for d, G, layout, combine in cases:
+        base = 1e4 if d == 64 else 1e6
+        offsets = [1 << i for i in range(11 if d == 64 else 17)]
+        B, S = 13, 40
+        lens = [0, 1, B, B + 1, S] + [int(x) for x in rng.integers(2, S + 1, 2)]
+        U = len(lens)
+        units = [_rand_unit(rng, d, G, S, layout, base) for _ in range(U)]
+        Kb = np.stack([u[3] for u in units])
+        Pb = np.stack([u[4] for u in units])
+        qm = np.stack([u[0] for u in units])
+        qn = np.stack([u[1] for u in units])
+        RR = np.stack([u[2] for u in units])
+        # t differs per unit: each unit's own t (its positions all lie below it)
+        tt = np.array([u[5] + 7 * i for i, u in enumerate(units)], np.int64)
+        kept, nk, zm = oracle.prune_batch(Kb, Pb, np.array(lens, np.int32), tt, qm, qn, RR, offsets, base, B,
+                                          layout, n_threads=2, want_zmax=True, L=L, combine=combine)
+        for u, n in enumerate(lens):
+            assert nk[u] == min(n, B), (d, G, combine, u, nk[u], n)
+            if n == 0:
+                continue
+            V = Kb[u, :n][::-1].copy()
+            one = oracle.prune_unit(Kb[u, :n], V, Pb[u, :n], int(tt[u]), qm[u], qn[u], RR[u], offsets, base, B,
+                                    layout, L=L, combine=combine)
+            assert np.array_equal(kept[u, :nk[u]], one["kept"]), (d, G, combine, u)
+            assert np.array_equal(zm[u, :n], one["zmax"]), (d, G, combine, u)
+
+
+def pin_select_f32(L, seed=13):
+    """Selection on fp32 max-z values: the B largest, ties to the lower slot, returned in
+    ascending slot order, checked against numpy's lexicographic sort on (-z, slot) and against
+    the fp64 selection of the same (exactly widened) values. Inputs carry many exact ties and
+    neighbours one fp32 ulp apart."""
+    rng = np.random.default_rng(seed)
+    for trial in range(40):
+        N = int(rng.integers(1, 300))
+        B = int(rng.integers(1, N + 20))
+        z = rng.integers(-6, 7, N).astype(np.float32) * np.float32(0.375)
+        bump = rng.random(N) < 0.3
+        z[bump] = np.nextafter(z[bump], np.float32(np.inf))
+        got = oracle.select(z, B, L=L)
+        assert got.dtype == np.int32
+        order = np.lexsort((np.arange(N), -z.astype(np.float64)))
+        want = np.sort(order[:min(N, B)])
+        assert np.array_equal(got, want), (N, B)
+        assert np.array_equal(got, oracle.select(z.astype(np.float64), B, L=L))
+
+
 def _calib_tokens(bands, d, layout):
     """[T][d] real vectors from [T][F][2] band samples, in the given rotary layout."""
     bands = np.asarray(bands, dtype=np.float64)
@@ -417,4 +474,5 @@ ALL_PINS = [pin_hand_examples, pin_rope_dot_closed_form, pin_positions_cancel,
             pin_t_shift_is_query_rotation, pin_norm_rotation_invariant_and_linear,
             pin_z_invariants, pin_scale_invariance, pin_select_brute_force, pin_compaction,
             pin_calibrate_hand_example, pin_calibrate_closed_forms, pin_calibrate_invariants,
-            pin_max_over_delta, pin_attention_special_cases, pin_attention_library]
+            pin_max_over_delta, pin_attention_special_cases, pin_attention_library,
+            pin_prune_batch_matches_units, pin_select_f32]

@@ -47,6 +47,12 @@ MUTANTS = {
     "attn_first_head_only": ("dot += bf16_value(q[(size_t)h * d + i]) * bf16_value(K[(size_t)j * d + i]);",
                              "dot += bf16_value(q[i]) * bf16_value(K[(size_t)j * d + i]);"),
     "attn_minus_logit": ("logit[j] = exp(logit[j] - top);", "logit[j] = exp(top - logit[j]);"),
+    "batch_qnorm_offset_drops_group": ("q_norm + (size_t)u * G * F", "q_norm + (size_t)u * F"),
+    "batch_keys_offset_by_length": ("K + (size_t)u * stride * d", "K + (size_t)u * N * d"),
+    "batch_kept_offset_by_count": ("tri_oracle_select(N, B, zm, kept_out + (size_t)u * B)",
+                                   "tri_oracle_select(N, B, zm, kept_out + (size_t)u * (N < B ? N : B))"),
+    "select_f32_truncates": ("for (int i = 0; i < N; ++i) z[i] = (double)zmax[i];",
+                             "for (int i = 0; i < N; ++i) z[i] = floor((double)zmax[i]);"),
 }
 
 

@@ -286,7 +286,7 @@ def make_cache(spec: CacheSpec, seed: int, device="cpu", lens=None, t=None,
         t_r = list(lens_r)
     maxlen = max(lens_r) if lens_r else 0
     omega = torch.as_tensor(rope_omega(d, spec.rope_base), device=device)
-    wdtype = torch.float64 if str(device) == "cpu" else torch.float32
+    wdtype = torch.float64  # keys drawn and rotated in fp64 on every device, then rounded RNE to bf16
     nan_bits = torch.tensor(BF16_NAN_BITS, dtype=torch.int16).view(torch.bfloat16)
 
     if spec.page_size:
