@@ -46,6 +46,7 @@ DEFAULT_WORKLOAD = "qwen3_8b_oneshot_32k_to_3072"
 METRIC = "KV tokens scored+pruned/s (Qwen3-8B shape); achieved HBM GB/s as % of B200 peak"
 UNIT = "keys/s"
 PEAK_FALLBACK_GBS = 6650.0
+NOMINAL_HBM_GBS = 8000.0  # B200 datasheet HBM3e bandwidth (the HGX figure is 7.7 TB/s)
 KERNEL_SOURCES = ["rope_aware_key_tri_b200/csrc/tri_kernel.cuh", "rope_aware_key_tri_b200/csrc/tri_api.cu"]
 KERNEL_NAME = "tri_fused_kernel"
 
@@ -109,6 +110,16 @@ def ncu_traffic(workload: str):
     if src != kernel_source_hash():
         return None
     return val
+
+
+def roofline_hbm(algorithmic_bytes: float, ms: float, traffic=None) -> dict:
+    """HBM roofline block: achieved algorithmic GB/s against the measured copy peak (the
+    fraction the targets are judged on) and, for context, against the datasheet figure."""
+    peak, kind = measured_peak()
+    achieved = algorithmic_bytes / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+            "traffic": traffic, "algorithmic_bytes": algorithmic_bytes, "peak_kind": f"{kind} (burst copy)",
+            "nominal_peak": NOMINAL_HBM_GBS, "frac_of_nominal": achieved / NOMINAL_HBM_GBS}
 
 
 def measured_peak():
@@ -206,6 +217,9 @@ def run_ours(args, rank, world, dist_mod):
         ctx.set_tuning(args.cluster_size, args.buffers)
     if args.combine != "mean":
         ctx.set_offset_combine(args.combine)
+    if args.engine != "auto":
+        ctx.set_score_engine(args.engine)
+    tensor_engine = args.combine == "max" or args.engine == "tensor" or (args.engine == "auto" and spec.group >= 8)
     lens_host = cache.lens_host.tolist()
     lens0 = cache.lens.clone()
     paged = cache.paged
@@ -282,18 +296,18 @@ def run_ours(args, rank, world, dist_mod):
     per_layer_scores = spec.batch * spec.n_kv_heads * cache.cap * spec.group * 4
     n_chunks = -(-spec.n_layers // max(1, min(spec.n_layers, (1 << 30) // per_layer_scores)))
     abytes = algorithmic_bytes(lens_host, spec.n_layers, spec.n_kv_heads, spec.head_dim, B)
-    peak, peak_kind = measured_peak()
-    achieved = abytes / (mean_ms / 1e3) / 1e9
     result = {
         "ms_per_step": mean_ms_max,
         "value": value,
         "ms_steps": {"min": min(ms), "median": statistics.median(ms), "max": max(ms)},
         "wall_ms_per_step_incl_restore": (wall1 - wall0) * 1e3 / args.steps,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": ncu_traffic(args.workload),
-                     "algorithmic_bytes": abytes, "peak_kind": f"{peak_kind} (burst copy)"},
+        "roofline": roofline_hbm(abytes, mean_ms, None if tensor_engine else ncu_traffic(args.workload)),
         "clocks": clk.summary(),
-        "gpu_launches": args.steps * (1 if args.combine == "mean" else 2 + 3 * n_chunks),
+        # fused engine: the validation kernel and the fused kernel; tensor-core engine (and the
+        # max mode): validation, prefix and phase kernels, then per chunk of layers the
+        # coefficient images, the tensor-core scoring and the fused select/compaction
+        "gpu_launches": args.steps * (3 + 3 * n_chunks if tensor_engine else 2),
+        "engine": "tensor cores + fused select" if tensor_engine else "fused (CUDA cores)",
         "keys_per_rank": keys_rank,
         "lens": lens_host,
     }
@@ -498,16 +512,13 @@ def run_calibrate(args):
     ms = statistics.median(times)
     rows = L * T
     nbytes = q.numel() * 2 + sum(x.numel() * 4 for x in out)
-    peak, kind = measured_peak()
-    achieved = nbytes / (ms * 1e-3) / 1e9
     res = {"metric": CAL_METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp64 sums", "data": "synthetic",
            "config": {"workload": "qwen3_8b_calibration_10k", "layers": L, "tokens": T, "q_heads": Hq,
                       "head_dim": d, "layout": "half",
                       "timed": "CUDA events around tri_calibrate_estimate (partial sums + means)"},
-           "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                        "traffic": None, "algorithmic_bytes": nbytes, "peak_kind": f"{kind} (burst copy)"},
+           "roofline": roofline_hbm(nbytes, ms),
            "clocks": clk.summary(), "gpu_launches": 2 * args.steps,
            "ms_steps": {"min": min(times), "median": ms, "max": max(times)}}
     if args.no_e2e:
@@ -678,8 +689,6 @@ def run_decode(args):
     row = d * 2
     units = L * batch * Hkv
     nbytes = cad * units * (2 * row + 4) + algorithmic_bytes([B + cad] * batch, L, Hkv, d, B)
-    peak, kind = measured_peak()
-    achieved = nbytes / (ms * 1e-3) / 1e9
     ctx.close()
     return {"metric": DEC_METRIC, "value": batch * cad / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
@@ -688,12 +697,139 @@ def run_decode(args):
                        "kv_heads": Hkv, "group": G, "head_dim": d, "batch": batch, "budget": B, "cadence": cad,
                        "timed": "CUDA events around one cycle: 128 tri_append (two CUDA-graph replays) + "
                                 "block-table copies + tri_prune"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                         "traffic": None, "algorithmic_bytes": nbytes, "peak_kind": f"{kind} (burst copy)"},
-            "clocks": clk.summary(), "gpu_launches": (2 * cad + 1) * args.steps,
+            "roofline": roofline_hbm(nbytes, ms),
+            # 128 appends of two launches each, the prune's validation and fused kernels
+            "clocks": clk.summary(), "gpu_launches": (2 * cad + 2) * args.steps,
             "ms_steps": {"min": min(times), "median": ms, "max": max(times)},
             "appends": "graph replay per 64-token page span" if graphs else (graph_note or "host-driven"),
             "host_driven_ms_per_step": statistics.median(times_host)}
+
+
+ATT_METRIC = "decode attention over the pruned cache: kept KV rows attended/s (Qwen3-8B shape)"
+
+
+def run_attend(args):
+    """One step = one decode step's attention over the whole pruned cache: every query head of
+    every unit attends over its kept rows (tri_decode_attention), CUDA events around the call on
+    its stream; a 256 MiB buffer is written between steps. The cache is the default workload
+    (one-shot 32K -> 3072 compression of the Qwen3-8B-shaped cache) after one tri_prune."""
+    import torch
+
+    import tri_synth as ts
+    from rope_aware_key_tri_b200 import tri
+    spec = workload_spec(args)
+    dev = torch.device("cuda", 0)
+    cache = ts.make_cache(spec, seed=1000, device=dev)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(spec.n_layers, spec.n_kv_heads, spec.group, spec.head_dim, spec.rope_base, spec.layout,
+                       cache.q_mean, cache.q_norm_mean, cache.R, cache.offsets)
+    ctx.prune(cache.K, cache.V, cache.pos, cache.lens, cache.t, spec.budget, block_table=cache.block_table)
+    st = ctx.get_error()
+    assert st[0] == tri.TRI_OK, st
+    lens = cache.lens_host.tolist()
+    gen = torch.Generator(device=dev).manual_seed(7)
+    q = (2.0 * torch.randn((spec.n_layers, spec.batch, spec.n_q_heads, spec.head_dim), generator=gen,
+                           device=dev)).to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        ctx.decode_attention(cache.K, cache.V, cache.lens, q, out=out, block_table=cache.block_table, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    times = []
+    with ClockSampler(0) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+    st = ctx.get_error()
+    assert st[0] == tri.TRI_OK, st
+    ms = sum(times) / len(times)
+    units = spec.n_layers * spec.batch * spec.n_kv_heads
+    rows = sum(lens) * spec.n_layers * spec.n_kv_heads
+    nbytes = rows * 2 * spec.head_dim * 2 + q.numel() * 2 + out.numel() * 4
+    # launches: validation, attention, and the chunk merge when units are split (two CTAs per SM)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    cap_u = cache.cap
+    cpu = max(1, min(-(-4 * sms * 2 // units), -(-cap_u // 256)))
+    res = {"metric": ATT_METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",
+           "config": {"workload": f"{args.workload} after one prune", "layers": spec.n_layers,
+                      "kv_heads": spec.n_kv_heads, "group": spec.group, "head_dim": spec.head_dim,
+                      "batch": spec.batch, "kept_rows_per_unit": sorted(set(lens))[:4],
+                      "l2": "256 MiB buffer written between steps; kept K+V %.2f GB" % (rows * 2 * spec.head_dim * 2 / 1e9),
+                      "timed": "CUDA events around tri_decode_attention"},
+           "roofline": roofline_hbm(nbytes, ms),
+           "clocks": clk.summary(), "gpu_launches": (3 if cpu > 1 else 2) * args.steps,
+           "ms_steps": {"min": min(times), "median": statistics.median(times), "max": max(times)}}
+    if not args.no_e2e:
+        # end to end: the step's queries from pinned host memory, the outputs back to the host
+        qh = q.cpu().pin_memory()
+        oh = torch.empty(out.shape, dtype=torch.float32).pin_memory()
+        e2e = []
+        for _ in range(3):
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            q.copy_(qh, non_blocking=True)
+            step()
+            oh.copy_(out, non_blocking=True)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            e2e.append(e0.elapsed_time(e1))
+        e = statistics.median(e2e[1:])
+        res["e2e"] = {"value": rows / (e * 1e-3), "unit": "rows/s", "ms_per_step": e,
+                      "h2d_bytes_per_step": q.numel() * 2, "d2h_bytes_per_step": out.numel() * 4, "steps": 2}
+    if not args.no_cpu:
+        res["cpu_baseline"] = time_oracle_attention(cache, spec, q)
+    ctx.close()
+    return res
+
+
+def time_oracle_attention(cache, spec, q, budget_s=10.0):
+    """The oracle's decode attention on whole units, threads over units (the C call releases the
+    interpreter lock), until about budget_s seconds of wall time."""
+    import numpy as np
+    from concurrent.futures import ThreadPoolExecutor
+
+    import oracle
+    cores = os.cpu_count() or 1
+    qb = q.view(torch_int16()).cpu().numpy().view(np.uint16)
+    G = spec.group
+    order = list(range(cache.n_units))
+    rows, done, t0 = 0, 0, time.perf_counter()
+
+    def one(u):
+        l, b, g = cache.unit_index(u)
+        n = int(cache.lens_host[b])
+        k, v, _ = cache.unit_rows(u)
+        oracle.decode_attention(qb[l, b, g * G:(g + 1) * G], k[:n], v[:n])
+        return n
+
+    with ThreadPoolExecutor(max_workers=cores) as ex:
+        while done < len(order) and time.perf_counter() - t0 < budget_s:
+            batch = order[done:done + cores]
+            rows += sum(ex.map(one, batch))
+            done += len(batch)
+    el = time.perf_counter() - t0
+    return {"value": rows / el, "unit": "rows/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {cache.n_units} units in full; {rows} rows in {el:.1f} s (incl. host copies)"}
+
+
+def torch_int16():
+    import torch
+    return torch.int16
 
 
 def main():
@@ -709,12 +845,15 @@ def main():
     ap.add_argument("--combine", default="mean", choices=["mean", "max"],
                     help="how the future offsets combine in the score (max: the tensor-core variant)")
     ap.add_argument("--buffers", type=int, default=0)
+    ap.add_argument("--engine", default="auto", choices=["auto", "cuda_cores", "tensor"],
+                    help="kernels that score the mean mode (auto: tensor cores at group 8)")
     ap.add_argument("--e2e-steps", type=int, default=2)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--path", default="prune", choices=["prune", "calibrate", "decode"],
+    ap.add_argument("--path", default="prune", choices=["prune", "calibrate", "decode", "attend"],
                     help="prune: the scoring-and-pruning pass (default); calibrate: the statistics estimator; "
-                         "decode: the decode loop's appends and prunes")
+                         "decode: the decode loop's appends and prunes; attend: decode attention over the "
+                         "pruned cache")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     if args.path == "calibrate":
@@ -722,6 +861,9 @@ def main():
         return
     if args.path == "decode":
         print(json.dumps(run_decode(args)), flush=True)
+        return
+    if args.path == "attend":
+        print(json.dumps(run_attend(args)), flush=True)
         return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -768,6 +910,7 @@ def main():
         "roofline": res["roofline"],
         "clocks": res["clocks"],
         "gpu_launches": res["gpu_launches"],
+        "engine": res["engine"],
         "ms_steps": res["ms_steps"],
         "wall_ms_per_step_incl_restore": res["wall_ms_per_step_incl_restore"],
     }

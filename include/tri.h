@@ -32,10 +32,19 @@
  *     calls return as soon as the work is enqueued (asynchronous).
  *   - Arguments are checked on the host before anything is launched; a failed
  *     check returns TRI_EINVAL (or TRI_ESTATE / TRI_EUNSUPPORTED) and launches
- *     nothing. Problems only the device can see (a length above the capacity,
- *     a page id outside the pool, a wait that ran out) are recorded in the
- *     context's device status word and read with tri_get_error; the affected
- *     sequence is left untouched. Kernels never trap.
+ *     nothing. Problems only the device can see are recorded in the context's
+ *     device status word and read with tri_get_error. Kernels never trap.
+ *     Two kinds:
+ *       sequence-level  a length above the capacity, a page id outside the pool, a
+ *                       cached position not below t. A validation kernel decides them
+ *                       before any unit of the call is touched, so every unit of the
+ *                       sequence is left untouched and lens_out[s] = lens[s].
+ *       unit-level      a bounded wait that ran out, or a selection that did not give
+ *                       exactly min(len, B) keys. Only that unit is left uncompacted; the
+ *                       sequence's other units are pruned and lens_out[s] = min(len, B), so
+ *                       the uncompacted unit then holds its first min(len, B) original rows
+ *                       (a consistent cache, ascending positions, but not the method's
+ *                       choice of keys). tri_get_failed_units lists such units.
  *   - A context is bound to one device and is not thread-safe: serialise calls
  *     that share a context. Calls that share a context but run on different
  *     streams must not overlap on the GPU (they share the status word, the
@@ -78,13 +87,21 @@ typedef enum {
     TRI_OFFSETS_MAX = 1    /* max over delta ([Deep-dive] §3.3 and its §4.2 scoring code) */
 } tri_offset_combine;
 
+/* Which kernels score the mean mode (tri_set_score_engine). */
+typedef enum {
+    TRI_ENGINE_AUTO = 0,        /* tensor cores at group 8, CUDA cores below (the default) */
+    TRI_ENGINE_CUDA_CORES = 1,  /* one fused launch: folded dot products on the CUDA cores */
+    TRI_ENGINE_TENSOR = 2       /* tcgen05 scoring kernel, then the fused select and compaction */
+} tri_score_engine;
+
 /* Device-side problem codes reported by tri_get_error in *detail_code. */
 enum {
     TRI_DEV_NONE = 0,
     TRI_DEV_LEN_GT_CAP = 1,   /* lens[s] < 0 or above the unit capacity */
     TRI_DEV_BAD_PAGE = 2,     /* a block-table entry outside [0, n_pages) */
-    TRI_DEV_TIMEOUT = 3,      /* a bounded wait on an asynchronous copy gave up */
-    TRI_DEV_INTERNAL = 4      /* the selection did not produce exactly min(len, B) keys */
+    TRI_DEV_TIMEOUT = 3,      /* a bounded wait on an asynchronous copy gave up (unit-level) */
+    TRI_DEV_INTERNAL = 4,     /* the selection did not produce exactly min(len, B) keys (unit-level) */
+    TRI_DEV_T_NOT_AFTER_POS = 5  /* a unit's last cached position is not below t (sequence-level) */
 };
 
 typedef struct tri_ctx tri_ctx;   /* opaque: device statistics, status word, counters */
@@ -126,7 +143,8 @@ typedef struct {
 } tri_kv;
 
 /* Create a context on CUDA device `device` (must be compute capability 10.0).
- * Allocates a few bytes of device memory (status word, completion counter). */
+ * Allocates about 16 KB of device memory (status word, completion counter, the list of units
+ * left uncompacted by unit-level failures). */
 TRI_API tri_status tri_create(tri_ctx **out, int device);
 
 /* Release the context and everything it allocated. NULL is accepted. */
@@ -200,7 +218,9 @@ TRI_API tri_status tri_calibrate_estimate(tri_ctx *ctx, const void *Q, int n_lay
 /*
  * Score every cached key and prune each unit to its top `budget` keys, in place.
  *   t       int32 [batch] device: current query position of each sequence; the
- *           future queries are at t + delta. Positions in the cache must be < t.
+ *           future queries are at t + delta. Positions in the cache must be < t: a
+ *           sequence with a unit whose last cached position is >= t is refused
+ *           (TRI_DEV_T_NOT_AFTER_POS, sequence-level).
  *   budget  B >= 1 keys kept per unit.
  * After the call (in stream order) slots [0, min(len, B)) of every unit hold the kept
  * K, V and position rows in ascending original order; slots at or beyond that are
@@ -233,11 +253,37 @@ TRI_API tri_status tri_prune_noalloc(tri_ctx *ctx, const tri_kv *kv, const int32
                                      void *stream);
 
 /*
+ * Decode attention over a (pruned) cache: the consumer of the compacted cache. For every query
+ * head h of every unit, out_h = sum_i softmax_i(q_h . k_i / sqrt(head_dim)) v_i over the unit's
+ * cached rows [0, lens[s]) (the page "TriAttention 深度解析：MIT韩松团队如何用三角函数让单卡
+ * 4090跑出百万Token上下文" writes this attention out in its section 二, TriAttention的核心发现).
+ * The query is post-RoPE like the stored keys, so each logit depends on the distance only and
+ * the kept keys' non-contiguous positions need no other treatment.
+ *   kv    the cache (dense or paged, as for tri_prune): K, V, lens, block table and layer range
+ *         are read; pos, lens_out are not used
+ *   q     bf16 [n_layers][batch][n_kv_heads*group][head_dim] device, 16-byte aligned: the
+ *         post-RoPE queries of the current decode step, one per query head
+ *   out   fp32 [n_layers][batch][n_kv_heads*group][head_dim] device, written
+ * Each K and V row is read once (HBM-bound); logits, the softmax and the weighted sum run in
+ * fp32 (exponentials in base 2 with the scale folded into the query). A sequence with lens 0
+ * gets zeros. Sequences refused by the sequence-level checks (length above the capacity, a page
+ * outside the pool; TRI_EDEVICE through tri_get_error) are not written. When there are too few
+ * units to fill the GPU, a unit's rows are split into chunks whose partial results a second
+ * launch merges; the partials live in the context's scratch, grown on demand (a synchronising
+ * cudaMalloc when a call needs more than any call before). Needs the statistics loaded (for
+ * n_kv_heads, group and head_dim). Errors: TRI_EINVAL, TRI_ESTATE, TRI_EUNSUPPORTED, TRI_ENOMEM,
+ * TRI_ECUDA.
+ */
+TRI_API tri_status tri_decode_attention(tri_ctx *ctx, const tri_kv *kv, const void *q, float *out, void *stream);
+
+/*
  * Debug / parity entry: score without pruning.
  *   raw   float [n_layers][batch][n_kv_heads*group][cap_u] or NULL: s_h(i) per query head
  *   zmax  float [n_layers][batch][n_kv_heads][cap_u] or NULL: max over the group of z_h(i)
  * where cap_u is cap (dense) or max_pages*page_size (paged), indexed by logical slot.
  * Slots at or beyond lens[s] are not written. The cache is not modified; lens_out is ignored.
+ * pos may be NULL here; when it is given, positions are checked against t as in tri_prune.
+ * Sequences refused by the sequence-level checks are not written at all.
  */
 TRI_API tri_status tri_score(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, float *raw, float *zmax,
                      void *stream);
@@ -249,6 +295,30 @@ TRI_API tri_status tri_score(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, f
  * (either out-pointer may be NULL).
  */
 TRI_API tri_status tri_get_error(tri_ctx *ctx, void *stream, int32_t *detail_code, int64_t *detail_unit);
+
+/*
+ * Synchronise `stream`, then read and clear the list of units that unit-level failures
+ * (TRI_DEV_TIMEOUT, TRI_DEV_INTERNAL) left uncompacted since the list was last read.
+ *   units     int32 host array of `capacity` entries, written with up to `capacity` unit
+ *             indices (as in tri_get_error), in no particular order; may be NULL when
+ *             capacity is 0
+ *   count     receives how many failures were recorded, which may exceed what was listed:
+ *             the device keeps the first 4096
+ * Device-detected sequence-level problems are not listed (tri_get_error reports them).
+ */
+TRI_API tri_status tri_get_failed_units(tri_ctx *ctx, void *stream, int32_t *units, int32_t capacity,
+                                        int32_t *count);
+
+/*
+ * Test hook for the failure path (not part of the paper's pass; off by default).
+ *   unit        index (as in tri_get_error) of a unit whose first key copy the scoring kernels
+ *               arm but never issue on the next calls, so that the wait for it runs out; -1 = off
+ *   wait_tries  tries of every bounded wait, about 1 ms each (0 = the default 1024)
+ * The withheld copy never lands, the wait gives up after wait_tries tries, the kernel records
+ * TRI_DEV_TIMEOUT and leaves the affected units uncompacted (unit-level failure); no copy is
+ * left in flight and nothing waits without bound.
+ */
+TRI_API tri_status tri_set_test_fault(tri_ctx *ctx, int64_t unit, int32_t wait_tries);
 
 /*
  * Launch-shape override for measurement and tests (not part of the paper's pass).
@@ -282,8 +352,29 @@ TRI_API tri_status tri_set_tuning(tri_ctx *ctx, int cluster_size, int buffers_pe
  * (42 KB at head_dim 128, group 4, 17 offsets) and small tables. tri_prune_noalloc supports
  * the mean only (TRI_EUNSUPPORTED in max mode). Errors: TRI_EINVAL (NULL context, unknown
  * mode).
+ * The max mode's scoring kernel runs one CTA per SM and allocates up to 512 columns of tensor
+ * memory per CTA with a blocking allocation: do not run it concurrently (on another stream)
+ * with other kernels that hold tensor memory on the same device, or its allocation may wait
+ * until they release theirs.
  */
 TRI_API tri_status tri_set_offset_combine(tri_ctx *ctx, int combine);
+
+/*
+ * Choose the kernels that score the mean mode on later tri_prune / tri_score calls (the max mode
+ * always uses the tensor cores; tri_prune_noalloc always the fused CUDA-core kernel).
+ *   TRI_ENGINE_CUDA_CORES  one fused launch per call: each key's folded dot products and norm
+ *                          terms on the CUDA cores (fp32), z-score, select and compaction on chip.
+ *   TRI_ENGINE_TENSOR      the tcgen05 kernel of the max mode with one column per head, whose
+ *                          coefficient is qbar A_f e^{i omega_f t} (the offset average folded in,
+ *                          as a hi + lo bf16 pair), writes the scores (group * 4 bytes per key,
+ *                          scratch grown on demand); then the fused kernel z-scores, selects and
+ *                          compacts. Worth it where the CUDA cores cannot keep up with HBM
+ *                          (group 8: about 13 flop per key byte).
+ *   TRI_ENGINE_AUTO        tensor cores at group 8, the fused kernel otherwise (the default).
+ * Results agree within the score tolerance (1e-4 of a head's largest score). Errors:
+ * TRI_EINVAL (NULL context, unknown engine).
+ */
+TRI_API tri_status tri_set_score_engine(tri_ctx *ctx, int engine);
 
 /* Tracing: tri_prune, tri_prune_noalloc, tri_score, tri_calibrate_estimate and tri_append each
  * mark their host-side span (argument checks and launches) with an NVTX range in the domain

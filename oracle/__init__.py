@@ -47,7 +47,7 @@ def _bind(L):
     L.tri_oracle_compact.argtypes = [i32, i32, P, P, P, P, P, P, P]
     L.tri_oracle_compact.restype = i32
     L.tri_oracle_prune_batch.argtypes = [i32, i32, i32, i32, i32, i32, f64, P, i32, P,
-                                         P, P, P, P, P, P, P, P, P, i32]
+                                         P, P, P, P, P, P, P, P, P, P, i32]
     L.tri_oracle_prune_batch.restype = i32
     L.tri_oracle_prune_batch_max.argtypes = L.tri_oracle_prune_batch.argtypes
     L.tri_oracle_prune_batch_max.restype = i32
@@ -144,11 +144,12 @@ def prune_unit(K_bits, V_bits, pos, t, q_mean, q_norm, R, offsets, base, B, layo
 
 
 def prune_batch(K_bits, pos, lens, t, q_mean, q_norm, R, offsets, base, B, layout=HALF,
-                n_threads=0, want_zmax=False, L=None, combine="mean"):
+                n_threads=0, want_zmax=False, L=None, combine="mean", want_scores=False):
     """Selection for many units at once (threads over units); combine "mean" or "max".
 
     K_bits [U][S][d] uint16, pos [U][S], lens [U], t [U], q_mean [U][G][d],
-    q_norm/R [U][G][d/2]. Returns (kept [U][B] int32, n_kept [U], zmax or None).
+    q_norm/R [U][G][d/2]. Returns (kept [U][B] int32, n_kept [U], zmax or None), and with
+    want_scores also the per-head scores s [U][G][S] as a fourth element.
     """
     L = L or lib()
     K_bits = _c(K_bits, np.uint16)
@@ -160,13 +161,14 @@ def prune_batch(K_bits, pos, lens, t, q_mean, q_norm, R, offsets, base, B, layou
     off = _c(offsets, np.int64)
     kept = np.zeros((U, B), np.int32); nk = np.zeros(U, np.int32)
     zm = np.zeros((U, S)) if want_zmax else None
+    sc = np.zeros((U, G, S)) if want_scores else None
     fn = {"mean": L.tri_oracle_prune_batch, "max": L.tri_oracle_prune_batch_max}[combine]
     rc = fn(U, S, int(B), d, G, layout, float(base), _p(off), len(off), _p(t),
             _p(q_mean), _p(q_norm), _p(R), _p(K_bits), _p(pos), _p(lens),
-            _p(zm), _p(kept), _p(nk), int(n_threads))
+            _p(sc), _p(zm), _p(kept), _p(nk), int(n_threads))
     if rc != 0:
         raise ValueError("tri_oracle_prune_batch rejected its arguments")
-    return kept, nk, zm
+    return (kept, nk, zm, sc) if want_scores else (kept, nk, zm)
 
 
 def calibrate(Q_bits, layout=HALF, L=None):

@@ -303,14 +303,15 @@ int tri_oracle_compact(int d, int M, const int32_t *kept,
  * The whole pass over a batch of units, units spread over threads.
  *   K [n_units][stride][d], pos [n_units][stride], lens [n_units] (<= stride),
  *   t [n_units], q_mean [n_units][G][d], q_norm / R [n_units][G][F].
- * Outputs (optional where marked): zmax [n_units][stride] (NULL ok),
- * kept [n_units][B], n_kept [n_units]. Returns 0, or -1 on a bad argument.
+ * Outputs (optional where marked): s [n_units][G][stride] per-head scores (NULL ok),
+ * zmax [n_units][stride] (NULL ok), kept [n_units][B], n_kept [n_units].
+ * Returns 0, or -1 on a bad argument.
  */
 static int prune_batch(int combine, int n_units, int stride, int B, int d, int G, int layout, double base,
                        const int64_t *offsets, int n_off, const int64_t *t,
                        const float *q_mean, const float *q_norm, const float *R,
                        const uint16_t *K, const int32_t *pos, const int32_t *lens,
-                       double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                       double *s_out, double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
                        int n_threads)
 {
     if (n_units < 0 || stride < 0 || B < 1 || d < 2 || G < 1)
@@ -333,6 +334,9 @@ static int prune_batch(int combine, int n_units, int stride, int B, int d, int G
                              pos + (size_t)u * stride, N, s, NULL, NULL);
         if (rc == 0) rc = tri_oracle_zmax(G, N, s, NULL, zm);
         if (rc == 0) {
+            if (s_out)
+                for (int h = 0; h < G; ++h)
+                    memcpy(s_out + ((size_t)u * G + h) * stride, s + (size_t)h * N, sizeof(double) * N);
             if (zmax_out) memcpy(zmax_out + (size_t)u * stride, zm, sizeof(double) * N);
             int m = tri_oracle_select(N, B, zm, kept_out + (size_t)u * B);
             n_kept_out[u] = m;
@@ -348,11 +352,11 @@ int tri_oracle_prune_batch(int n_units, int stride, int B, int d, int G, int lay
                            const int64_t *offsets, int n_off, const int64_t *t,
                            const float *q_mean, const float *q_norm, const float *R,
                            const uint16_t *K, const int32_t *pos, const int32_t *lens,
-                           double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                           double *s_out, double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
                            int n_threads)
 {
     return prune_batch(TRI_ORACLE_MEAN_OVER_DELTA, n_units, stride, B, d, G, layout, base, offsets, n_off, t,
-                       q_mean, q_norm, R, K, pos, lens, zmax_out, kept_out, n_kept_out, n_threads);
+                       q_mean, q_norm, R, K, pos, lens, s_out, zmax_out, kept_out, n_kept_out, n_threads);
 }
 
 /* The same selection with the offsets combined by the maximum (tri_oracle_unit_scores_max). */
@@ -360,11 +364,11 @@ int tri_oracle_prune_batch_max(int n_units, int stride, int B, int d, int G, int
                                const int64_t *offsets, int n_off, const int64_t *t,
                                const float *q_mean, const float *q_norm, const float *R,
                                const uint16_t *K, const int32_t *pos, const int32_t *lens,
-                               double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
+                               double *s_out, double *zmax_out, int32_t *kept_out, int32_t *n_kept_out,
                                int n_threads)
 {
     return prune_batch(TRI_ORACLE_MAX_OVER_DELTA, n_units, stride, B, d, G, layout, base, offsets, n_off, t,
-                       q_mean, q_norm, R, K, pos, lens, zmax_out, kept_out, n_kept_out, n_threads);
+                       q_mean, q_norm, R, K, pos, lens, s_out, zmax_out, kept_out, n_kept_out, n_threads);
 }
 
 /*

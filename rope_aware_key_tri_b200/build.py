@@ -14,7 +14,7 @@ LIBDIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIBDIR, "libtri_b200.so")
 SOURCES = [os.path.join(CSRC, "tri_api.cu")]
 EXPORTS = os.path.join(CSRC, "exports.map")
-DEPS = SOURCES + [os.path.join(CSRC, "tri_kernel.cuh"), os.path.join(CSRC, "tri_calib.cuh"), os.path.join(CSRC, "tri_append.cuh"), os.path.join(CSRC, "tri_maxdelta.cuh"), os.path.join(ROOT, "include", "tri.h"), EXPORTS]
+DEPS = SOURCES + [os.path.join(CSRC, "tri_kernel.cuh"), os.path.join(CSRC, "tri_calib.cuh"), os.path.join(CSRC, "tri_append.cuh"), os.path.join(CSRC, "tri_maxdelta.cuh"), os.path.join(CSRC, "tri_attend.cuh"), os.path.join(ROOT, "include", "tri.h"), EXPORTS]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -25,6 +25,7 @@
 #include "tri_calib.cuh"
 #include "tri_append.cuh"
 #include "tri_maxdelta.cuh"
+#include "tri_attend.cuh"
 
 struct tri_ctx {
     int device = -1;
@@ -38,8 +39,10 @@ struct tri_ctx {
     float *d_w = nullptr;
     double2 *d_qbar = nullptr;      // [L][Hq][F] qbar itself (the max-over-offsets mode)
     int64_t *d_offsets = nullptr;   // [n_off]
+    int64_t *d_zero_offset = nullptr;  // [1] = {0}: the tensor-core mean mode's single column
     int n_off = 0;
     int combine = TRI_OFFSETS_MEAN;
+    int engine = TRI_ENGINE_AUTO;     // which kernels score the mean mode (tri_set_score_engine)
     // scratch of the max-over-offsets mode, grown on demand
     float *d_pre = nullptr;
     size_t pre_bytes = 0;
@@ -51,11 +54,21 @@ struct tri_ctx {
     size_t tile_prefix_bytes = 0;
     int32_t *d_unit_fail = nullptr;
     size_t unit_fail_bytes = 0;
+    // chunk partials of tri_decode_attention, grown on demand
+    float *d_att_part = nullptr;
+    size_t att_part_bytes = 0;
     // device bookkeeping
     unsigned long long *d_status = nullptr;
     unsigned int *d_counter = nullptr;
-    int32_t *d_seq_bad = nullptr;
+    int32_t *d_seq_bad = nullptr;    // per-sequence verdict of the validation kernel
     int seq_bad_cap = 0;
+    int32_t *d_append_bad = nullptr; // per-sequence refusal flags of tri_append
+    int append_bad_cap = 0;
+    unsigned *d_fail_count = nullptr;  // units left uncompacted by a unit-level failure ...
+    int32_t *d_fail_units = nullptr;   // ... the first kFailCap of them
+    // test hook (tri_set_test_fault): bounded waits' tries and the unit whose copy is withheld
+    int wait_tries = tri::kWaitTries;
+    long long inject_unit = -1;
     float *d_scratch = nullptr;      // per-cluster score slots of the persistent grid
     size_t scratch_bytes = 0;
     // tuning (0 = automatic)
@@ -127,6 +140,8 @@ void free_stats(tri_ctx *c) {
     cudaFree(c->d_w);
     cudaFree(c->d_qbar);
     cudaFree(c->d_offsets);
+    cudaFree(c->d_zero_offset);
+    c->d_zero_offset = nullptr;
     c->d_omega = nullptr;
     c->d_Qc = nullptr;
     c->d_w = nullptr;
@@ -149,12 +164,14 @@ KernelFn pick_pre_kernel(int D, int G) {
 using MxImageFn = void (*)(const tri::MxArgs);
 using MxScoreFn = void (*)(const CUtensorMap, const tri::MxArgs);
 
-bool pick_mx(int D, int G, int layout, MxImageFn *img, MxScoreFn *score) {
-#define TRI_MX_CASE(DD, GG, LL)                                  \
-    if (D == DD && G == GG && layout == LL) {                    \
-        *img = &tri::tri_mx_image_kernel<DD, GG, LL>;            \
-        *score = &tri::tri_mx_score_kernel<DD, GG, LL>;          \
-        return true;                                             \
+bool pick_mx(int D, int G, int layout, int noffp, MxImageFn *img, MxScoreFn *score) {
+#define TRI_MX_CASE(DD, GG, LL)                                                        \
+    if (D == DD && G == GG && layout == LL) {                                          \
+        *img = &tri::tri_mx_image_kernel<DD, GG, LL>;                                  \
+        *score = noffp == 1    ? &tri::tri_mx_score_kernel<DD, GG, LL, 1>              \
+                 : noffp == 17 ? &tri::tri_mx_score_kernel<DD, GG, LL, 17>             \
+                               : &tri::tri_mx_score_kernel<DD, GG, LL, 32>;            \
+        return noffp == 1 || noffp == 17 || noffp == 32;                               \
     }
     TRI_MX_CASE(64, 1, 0) TRI_MX_CASE(64, 2, 0) TRI_MX_CASE(64, 4, 0) TRI_MX_CASE(64, 8, 0)
     TRI_MX_CASE(64, 1, 1) TRI_MX_CASE(64, 2, 1) TRI_MX_CASE(64, 4, 1) TRI_MX_CASE(64, 8, 1)
@@ -192,6 +209,9 @@ struct Plan {
     int cs = 0, nslot = 0, kpc = 0, n_clusters = 0, extra = 0;
     size_t smem = 0;
 };
+
+// Capacity of the device list of units that a unit-level failure left uncompacted.
+constexpr int kFailCap = 4096;
 
 // Live score slots should stay well inside the 126 MB L2 so that the scores written during
 // streaming are read back from L2.
@@ -368,6 +388,7 @@ tri_status check_call(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t bu
     } else {
         if (!kv->K || !kv->lens) return TRI_EINVAL;
         if (!aligned(kv->K, 16) || !is_device_ptr(kv->K)) return TRI_EINVAL;
+        if (kv->pos && (!aligned(kv->pos, 4) || !is_device_ptr(kv->pos))) return TRI_EINVAL;
         if (raw && (!aligned(raw, 4) || !is_device_ptr(raw))) return TRI_EINVAL;
         if (zmax && (!aligned(zmax, 4) || !is_device_ptr(zmax))) return TRI_EINVAL;
     }
@@ -381,24 +402,72 @@ tri_status check_call(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t bu
     return TRI_OK;
 }
 
-tri_status ensure_seq_bad(tri_ctx *c, int batch) {
-    if (batch <= c->seq_bad_cap) return TRI_OK;
-    cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
-    c->d_seq_bad = nullptr;
-    c->seq_bad_cap = 0;
-    if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ENOMEM;
-    if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ECUDA;
-    c->seq_bad_cap = batch;
+// Grow a per-sequence int32 array of the context to `batch` entries (zeroed).
+tri_status ensure_flags(int32_t **p, int *cap, int batch) {
+    if (batch <= *cap) return TRI_OK;
+    cudaFree(*p);  // synchronises the device: no call still uses the old flags
+    *p = nullptr;
+    *cap = 0;
+    if (cudaMalloc(p, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ENOMEM;
+    if (cudaMemset(*p, 0, sizeof(int32_t) * batch) != cudaSuccess) return TRI_ECUDA;
+    *cap = batch;
+    return TRI_OK;
+}
+
+tri_status ensure_seq_bad(tri_ctx *c, int batch) { return ensure_flags(&c->d_seq_bad, &c->seq_bad_cap, batch); }
+
+// Arguments shared by the validation kernel and the fused kernel of one call.
+tri::Args base_args(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, int mode, long long cap_u,
+                    int32_t *seq_bad) {
+    const bool paged = kv->block_table != nullptr;
+    tri::Args a;
+    std::memset(&a, 0, sizeof a);
+    a.K = static_cast<uint16_t *>(kv->K);
+    a.V = static_cast<uint16_t *>(kv->V);
+    a.pos = kv->pos;
+    a.lens = kv->lens;
+    a.block_table = kv->block_table;
+    a.t = t;
+    a.batch = kv->batch;
+    a.n_kv = c->Hkv;
+    a.cap_u = (int)cap_u;
+    a.paged = paged ? 1 : 0;
+    a.page_size = paged ? kv->page_size : 0;
+    a.max_pages = paged ? kv->max_pages : 0;
+    a.n_pages = paged ? kv->n_pages : 0;
+    a.layer_begin = kv->layer_begin;
+    a.budget = mode == tri::kModePrune ? budget : 0x7fffffff;
+    a.n_units = (int)((long long)kv->n_layers * kv->batch * c->Hkv);
+    a.mode = mode;
+    a.status = c->d_status;
+    a.counter = c->d_counter;
+    a.seq_bad = seq_bad;
+    a.wait_tries = c->wait_tries;
+    a.inject_unit = c->inject_unit;
+    a.fail_count = c->d_fail_count;
+    a.fail_units = c->d_fail_units;
+    a.fail_cap = kFailCap;
+    return a;
+}
+
+// The sequence-level checks of a call (tri::tri_validate_kernel), before any unit is touched:
+// seq_bad[s] receives each sequence's verdict. Positions are checked against t when the call
+// passes them (tri_score may not).
+tri_status launch_validate(tri_ctx *c, const tri_kv *kv, const int32_t *t, int mode, long long cap_u,
+                           int32_t *seq_bad, void *stream) {
+    const tri::Args a = base_args(c, kv, t, 0, mode, cap_u, seq_bad);
+    tri::tri_validate_kernel<<<(unsigned)kv->batch, tri::kValidateThreads, 0, static_cast<cudaStream_t>(stream)>>>(a);
+    const cudaError_t ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(validate)");
     return TRI_OK;
 }
 
 // One launch of the fused kernel `fn` over the units of kv. pre / unit_fail: precomputed
 // scores (the PRE variant) or null; lens_out: where the last CTA publishes the new lengths
-// (null: not in this launch); seq_bad: refusal flags (null: none kept).
+// (null: not in this launch); seq_bad: the validation kernel's per-sequence verdicts.
 tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw,
                         float *zmax, int mode, long long cap_u, const float *pre, const int32_t *unit_fail,
                         long long unit_base, int32_t *lens_out, int32_t *seq_bad, void *stream) {
-    const bool paged = kv->block_table != nullptr;
     const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
@@ -419,40 +488,19 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
         c->scratch_bytes = need;
     }
 
-    tri::Args a;
-    std::memset(&a, 0, sizeof a);
-    a.K = static_cast<uint16_t *>(kv->K);
-    a.V = static_cast<uint16_t *>(kv->V);
-    a.pos = kv->pos;
-    a.lens = kv->lens;
+    tri::Args a = base_args(c, kv, t, budget, mode, cap_u, seq_bad);
     a.lens_out = mode == tri::kModePrune ? lens_out : nullptr;
-    a.block_table = kv->block_table;
-    a.t = t;
-    a.batch = kv->batch;
-    a.n_kv = c->Hkv;
-    a.cap_u = (int)cap_u;
-    a.paged = paged ? 1 : 0;
-    a.page_size = paged ? kv->page_size : 0;
-    a.max_pages = paged ? kv->max_pages : 0;
-    a.n_pages = paged ? kv->n_pages : 0;
-    a.layer_begin = kv->layer_begin;
-    a.budget = mode == tri::kModePrune ? budget : 0x7fffffff;
     a.omega = c->d_omega;
     a.Qc = c->d_Qc;
     a.w = c->d_w;
     a.raw = raw;
     a.zmax = zmax;
-    a.mode = mode;
     a.cs = plan.cs;
     a.kpc_max = plan.kpc;
     a.nslot = plan.nslot;
     a.ring_extra = plan.extra;
-    a.n_units = (int)n_units;
     a.scratch = c->d_scratch;
     a.slot_floats = slot_floats;
-    a.status = c->d_status;
-    a.counter = c->d_counter;
-    a.seq_bad = mode == tri::kModePrune ? seq_bad : nullptr;
     a.pre = pre;
     a.unit_fail = unit_fail;
     a.unit_base = unit_base;
@@ -509,19 +557,23 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 // Scores held for at most this many bytes at a time; longer calls run in chunks of layers.
 constexpr size_t kMaxPreBytes = size_t(1) << 30;
 
-// The max-over-offsets mode: per chunk of layers, the tensor-core scoring kernel writes every
-// unit's scores, then the fused kernel's PRE variant z-scores, selects and compacts.
+// The tensor-core engine: per chunk of layers, the tcgen05 scoring kernel writes every unit's
+// scores, then the fused kernel's PRE variant z-scores, selects and compacts. With the offsets
+// combined by the maximum every (head, offset) is a column; for the mean (mean_tc) a head has
+// one column whose coefficient carries the folded offset average, qbar A_f e^{i omega_f t}.
 tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
-                   int mode, long long cap_u, void *stream) {
+                   int mode, long long cap_u, void *stream, bool mean_tc = false) {
     const int D = c->D, G = c->G, F = D / 2, Hkv = c->Hkv, Hq = Hkv * G;
-    if (G * c->n_off > 256) {
+    const int noffp = mean_tc ? 1 : tri::mx_noff_pad(c->n_off);
+    if ((!mean_tc && c->n_off > 32) || G * noffp > 256) {
         std::snprintf(c->last_error, sizeof c->last_error,
-                      "max over offsets: group * n_offsets = %d exceeds the 256 columns of one MMA", G * c->n_off);
+                      "max over offsets: %d offsets (padded to %d) for a group of %d exceed the 256 columns of one "
+                      "MMA (at most 32 offsets)", c->n_off, noffp, G);
         return TRI_EUNSUPPORTED;
     }
     MxImageFn img_fn = nullptr;
     MxScoreFn score_fn = nullptr;
-    if (!pick_mx(D, G, c->layout, &img_fn, &score_fn)) return TRI_EUNSUPPORTED;
+    if (!pick_mx(D, G, c->layout, noffp, &img_fn, &score_fn)) return TRI_EUNSUPPORTED;
     KernelFn fused = pick_pre_kernel(D, G);
     if (!fused) return TRI_EUNSUPPORTED;
     PFN_cuTensorMapEncodeTiled_v12000 encode = tensor_map_encoder();
@@ -530,8 +582,7 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
         return TRI_ECUDA;
     }
     const bool paged = kv->block_table != nullptr;
-    const int ncol = tri::mx_ncol(G, c->n_off);
-    const int acc_cols = tri::mx_acc_cols(ncol);
+    const int ncol = tri::mx_ncol(G, noffp);
     const unsigned img_bytes = tri::mx_image_bytes(D, G, ncol);
     int piece_rows = 64;
     if (paged) {
@@ -573,7 +624,8 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
                    "cudaMalloc(unit flags)")) != TRI_OK)
         return st;
     const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
-    if (finalize && (st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+    if ((st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+    if ((st = launch_validate(c, kv, t, mode, cap_u, c->d_seq_bad, stream)) != TRI_OK) return st;
 
     tri::MxArgs m;
     std::memset(&m, 0, sizeof m);
@@ -588,14 +640,14 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
     m.max_pages = paged ? kv->max_pages : 0;
     m.n_pages = paged ? kv->n_pages : 0;
     m.min_len = mode == tri::kModePrune ? budget : 0;
-    m.n_off = c->n_off;
+    m.n_off = mean_tc ? 1 : c->n_off;
+    m.noffp = noffp;
     m.ncol = ncol;
-    m.acc_cols = acc_cols;
     m.nst = nst;
     m.piece_rows = piece_rows;
-    m.qbar = c->d_qbar;
+    m.qbar = mean_tc ? c->d_Qc : c->d_qbar;
     m.omega = c->d_omega;
-    m.offsets = c->d_offsets;
+    m.offsets = mean_tc ? c->d_zero_offset : c->d_offsets;
     m.w = c->d_w;
     m.phase = c->d_phase;
     m.image = c->d_image;
@@ -603,10 +655,13 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
     m.pre = c->d_pre;
     m.unit_fail = c->d_unit_fail;
     m.status = c->d_status;
+    m.seq_bad = c->d_seq_bad;
+    m.wait_tries = c->wait_tries;
+    m.inject_unit = c->inject_unit;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
     tri::tri_mx_prefix_kernel<<<1, 32, 0, cs>>>(m);
-    const long long n_ph = (long long)kv->batch * c->n_off * F;
+    const long long n_ph = (long long)kv->batch * m.n_off * F;
     tri::tri_mx_phase_kernel<<<(unsigned)((n_ph + 255) / 256), 256, 0, cs>>>(m, F);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(prefix, phase)");
@@ -653,11 +708,20 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
         if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx(score)");
         const bool last = lr0 + nl == kv->n_layers;
         st = launch_fused(c, fused, &sub, t, budget, raw_c, zmax_c, mode, cap_u, c->d_pre, c->d_unit_fail,
-                          m.unit_base, (finalize && last) ? kv->lens_out : nullptr,
-                          finalize ? c->d_seq_bad : nullptr, stream);
+                          m.unit_base, (finalize && last) ? kv->lens_out : nullptr, c->d_seq_bad, stream);
         if (st != TRI_OK) return st;
     }
     return TRI_OK;
+}
+
+// The mean mode's engine: the fused CUDA-core kernel, or the tensor-core scoring kernel followed
+// by the fused kernel's select and compaction. Automatic: tensor cores at group 8, where the
+// folded dot products and norm weights of a key (about 13 flop per key byte) exceed what the
+// CUDA cores deliver at the HBM rate; the fused kernel below that (one launch, no score traffic).
+bool use_tensor_engine(const tri_ctx *c) {
+    if (c->engine == TRI_ENGINE_TENSOR) return true;
+    if (c->engine == TRI_ENGINE_CUDA_CORES) return false;
+    return c->G >= 8;
 }
 
 tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw, float *zmax,
@@ -666,12 +730,14 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     tri_status st = check_call(c, kv, t, budget, raw, zmax, mode, &cap_u);
     if (st != TRI_OK) return st;
     if (c->combine == TRI_OFFSETS_MAX) return run_max(c, kv, t, budget, raw, zmax, mode, cap_u, stream);
+    if (use_tensor_engine(c)) return run_max(c, kv, t, budget, raw, zmax, mode, cap_u, stream, true);
     KernelFn fn = pick_kernel(c->D, c->G, c->layout);
     if (!fn) return TRI_EUNSUPPORTED;
     const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
-    if (finalize && (st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+    if ((st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
+    if ((st = launch_validate(c, kv, t, mode, cap_u, c->d_seq_bad, stream)) != TRI_OK) return st;
     return launch_fused(c, fn, kv, t, budget, raw, zmax, mode, cap_u, nullptr, nullptr, 0,
-                        finalize ? kv->lens_out : nullptr, finalize ? c->d_seq_bad : nullptr, stream);
+                        finalize ? kv->lens_out : nullptr, c->d_seq_bad, stream);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -789,45 +855,21 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     }
     const int n_clusters = (int)std::min<long long>(plan.n_clusters, slots);
 
-    const bool finalize = kv->lens_out != nullptr;
-    if (finalize) {
-        // the refusal flags must start at zero; they keep whatever the last call left
-        ce = cudaMemsetAsync(sym.seq_bad, 0, sizeof(int32_t) * kv->batch, static_cast<cudaStream_t>(stream));
-        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaMemsetAsync(flags)");
-    }
+    // the per-sequence verdicts go to the fixed flag array, written whole by the validation kernel
+    st = launch_validate(c, kv, t, tri::kModePrune, cap_u, sym.seq_bad, stream);
+    if (st != TRI_OK) return st;
 
-    tri::Args a;
-    std::memset(&a, 0, sizeof a);
-    a.K = static_cast<uint16_t *>(kv->K);
-    a.V = static_cast<uint16_t *>(kv->V);
-    a.pos = kv->pos;
-    a.lens = kv->lens;
-    a.lens_out = finalize ? kv->lens_out : nullptr;
-    a.block_table = kv->block_table;
-    a.t = t;
-    a.batch = kv->batch;
-    a.n_kv = c->Hkv;
-    a.cap_u = (int)cap_u;
-    a.paged = paged ? 1 : 0;
-    a.page_size = paged ? kv->page_size : 0;
-    a.max_pages = paged ? kv->max_pages : 0;
-    a.n_pages = paged ? kv->n_pages : 0;
-    a.layer_begin = kv->layer_begin;
-    a.budget = budget;
+    tri::Args a = base_args(c, kv, t, budget, tri::kModePrune, cap_u, sym.seq_bad);
+    a.lens_out = kv->lens_out;
     a.omega = c->d_omega;
     a.Qc = c->d_Qc;
     a.w = c->d_w;
-    a.mode = tri::kModePrune;
     a.cs = plan.cs;
     a.kpc_max = plan.kpc;
     a.nslot = plan.nslot;
     a.ring_extra = plan.extra;
-    a.n_units = (int)n_units;
     a.scratch = sym.scratch;
     a.slot_floats = slot_floats;
-    a.status = c->d_status;
-    a.counter = c->d_counter;
-    a.seq_bad = finalize ? sym.seq_bad : nullptr;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
@@ -862,6 +904,118 @@ bool pick_calib(int D, int layout, CalPartialFn *p, CalFinalFn *f) {
     return false;
 }
 
+using AttFn = void (*)(const tri::AttArgs);
+
+bool pick_attend(int D, int G, AttFn *main_fn, AttFn *combine_fn) {
+#define TRI_ATT_CASE(DD, GG)                                      \
+    if (D == DD && G == GG) {                                     \
+        *main_fn = &tri::tri_attend_kernel<DD, GG>;               \
+        *combine_fn = &tri::tri_attend_combine_kernel<DD, GG>;    \
+        return true;                                              \
+    }
+    TRI_ATT_CASE(64, 1) TRI_ATT_CASE(64, 2) TRI_ATT_CASE(64, 4) TRI_ATT_CASE(64, 8)
+    TRI_ATT_CASE(128, 1) TRI_ATT_CASE(128, 2) TRI_ATT_CASE(128, 4) TRI_ATT_CASE(128, 8)
+#undef TRI_ATT_CASE
+    return false;
+}
+
+tri_status run_attend(tri_ctx *c, const tri_kv *kv, const void *q, float *out, void *stream) {
+    if (!c || !kv || !q || !out) return TRI_EINVAL;
+    if (!c->loaded) return TRI_ESTATE;
+    if (kv->batch < 1 || kv->n_layers < 1 || kv->layer_begin < 0 || kv->layer_begin + kv->n_layers > c->L)
+        return TRI_EINVAL;
+    const bool paged = kv->block_table != nullptr;
+    long long cap_u;
+    if (paged) {
+        if (kv->page_size < 16 || kv->page_size % 16 != 0 || kv->max_pages < 1 || kv->n_pages < 1)
+            return TRI_EINVAL;
+        cap_u = (long long)kv->page_size * kv->max_pages;
+    } else {
+        if (kv->cap < 1) return TRI_EINVAL;
+        cap_u = kv->cap;
+    }
+    if (cap_u > (1LL << 30)) return TRI_EUNSUPPORTED;
+    if (!kv->K || !kv->V || !kv->lens) return TRI_EINVAL;
+    if (!aligned(kv->K, 16) || !aligned(kv->V, 16) || !aligned(q, 16) || !aligned(out, 4) ||
+        !aligned(kv->lens, 4))
+        return TRI_EINVAL;
+    if (!is_device_ptr(kv->K) || !is_device_ptr(kv->V) || !is_device_ptr(q) || !is_device_ptr(out) ||
+        !is_device_ptr(kv->lens))
+        return TRI_EINVAL;
+    if (paged && (!is_device_ptr(kv->block_table) || !aligned(kv->block_table, 4))) return TRI_EINVAL;
+    AttFn fn = nullptr, comb = nullptr;
+    if (!pick_attend(c->D, c->G, &fn, &comb)) return TRI_EUNSUPPORTED;
+    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
+    if (n_units > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+    cudaError_t ce = cudaSetDevice(c->device);
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
+
+    // launch shape: the deepest per-warp ring (3 stages at most) that keeps two CTAs per SM
+    int nslot = 3, per_sm = 0;
+    for (; nslot >= 1; --nslot) {
+        const size_t smem = tri::att_smem_bytes(c->D, c->G, nslot);
+        ce = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute(attend)");
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::kAttThreads, smem) != cudaSuccess) {
+            cudaGetLastError();
+            per_sm = 0;
+        }
+        if (per_sm >= 2 || nslot == 1) break;
+    }
+    if (per_sm < 1) return TRI_EUNSUPPORTED;
+    // chunks per unit: split the units' rows only when there are too few units for four waves
+    const long long target = 4LL * c->sm_count * per_sm;
+    long long cpu = (target + n_units - 1) / n_units;
+    cpu = std::max<long long>(1, std::min<long long>(cpu, (cap_u + 255) / 256));
+    if (n_units * cpu > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+
+    tri_status st = ensure_seq_bad(c, kv->batch);
+    if (st != TRI_OK) return st;
+    if (cpu > 1) {
+        const size_t need = (size_t)n_units * cpu * c->G * (c->D + 2) * sizeof(float);
+        if ((st = grow(c, &c->d_att_part, &c->att_part_bytes, need, "cudaMalloc(attention partials)")) != TRI_OK)
+            return st;
+    }
+    // sequence-level checks (length, pages; no positions: the attention does not read them)
+    tri_kv chk = *kv;
+    chk.pos = nullptr;
+    if ((st = launch_validate(c, &chk, nullptr, tri::kModeScore, cap_u, c->d_seq_bad, stream)) != TRI_OK) return st;
+
+    tri::AttArgs a;
+    std::memset(&a, 0, sizeof a);
+    a.K = static_cast<const uint16_t *>(kv->K);
+    a.V = static_cast<const uint16_t *>(kv->V);
+    a.q = static_cast<const uint16_t *>(q);
+    a.out = out;
+    a.part = c->d_att_part;
+    a.lens = kv->lens;
+    a.block_table = kv->block_table;
+    a.seq_bad = c->d_seq_bad;
+    a.batch = kv->batch;
+    a.n_kv = c->Hkv;
+    a.cap_u = (int)cap_u;
+    a.paged = paged ? 1 : 0;
+    a.page_size = paged ? kv->page_size : 0;
+    a.max_pages = paged ? kv->max_pages : 0;
+    a.n_pages = paged ? kv->n_pages : 0;
+    a.n_units = (int)n_units;
+    a.cpu = (int)cpu;
+    a.nslot = nslot;
+    a.qscale = (float)(1.4426950408889634 / std::sqrt((double)c->D));
+    a.status = c->d_status;
+    a.wait_tries = c->wait_tries;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    fn<<<(unsigned)(n_units * cpu), tri::kAttThreads, tri::att_smem_bytes(c->D, c->G, nslot), cs>>>(a);
+    ce = cudaGetLastError();
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(attend)");
+    if (cpu > 1) {
+        comb<<<(unsigned)n_units, 256, 0, cs>>>(a);
+        ce = cudaGetLastError();
+        if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(attend combine)");
+    }
+    return TRI_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -885,12 +1039,15 @@ tri_status tri_create(tri_ctx **out, int device) {
     c->sm_count = p.multiProcessorCount;
     c->max_smem_optin = (int)p.sharedMemPerBlockOptin;
     if (cudaMalloc(&c->d_status, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMalloc(&c->d_counter, sizeof(unsigned int)) != cudaSuccess) {
+        cudaMalloc(&c->d_counter, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMalloc(&c->d_fail_count, sizeof(unsigned)) != cudaSuccess ||
+        cudaMalloc(&c->d_fail_units, sizeof(int32_t) * kFailCap) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ENOMEM;
     }
     if (cudaMemset(c->d_status, 0, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMemset(c->d_counter, 0, sizeof(unsigned int)) != cudaSuccess) {
+        cudaMemset(c->d_counter, 0, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(c->d_fail_count, 0, sizeof(unsigned)) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ECUDA;
     }
@@ -905,12 +1062,16 @@ tri_status tri_destroy(tri_ctx *c) {
     cudaFree(c->d_status);
     cudaFree(c->d_counter);
     cudaFree(c->d_seq_bad);
+    cudaFree(c->d_append_bad);
+    cudaFree(c->d_fail_count);
+    cudaFree(c->d_fail_units);
     cudaFree(c->d_scratch);
     cudaFree(c->d_pre);
     cudaFree(c->d_image);
     cudaFree(c->d_phase);
     cudaFree(c->d_tile_prefix);
     cudaFree(c->d_unit_fail);
+    cudaFree(c->d_att_part);
     delete c;
     return TRI_OK;
 }
@@ -963,7 +1124,8 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
         cudaMalloc(&c->d_Qc, sizeof(double2) * nb) != cudaSuccess ||
         cudaMalloc(&c->d_w, sizeof(float) * nb) != cudaSuccess ||
         cudaMalloc(&c->d_qbar, sizeof(double2) * nb) != cudaSuccess ||
-        cudaMalloc(&c->d_offsets, sizeof(int64_t) * n_offsets) != cudaSuccess) {
+        cudaMalloc(&c->d_offsets, sizeof(int64_t) * n_offsets) != cudaSuccess ||
+        cudaMalloc(&c->d_zero_offset, sizeof(int64_t)) != cudaSuccess) {
         free_stats(c);
         return TRI_ENOMEM;
     }
@@ -971,7 +1133,8 @@ tri_status tri_calibrate_load(tri_ctx *c, int n_layers, int n_kv_heads, int grou
         cudaMemcpy(c->d_Qc, Qc.data(), sizeof(double2) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->d_w, w.data(), sizeof(float) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
         cudaMemcpy(c->d_qbar, qbar.data(), sizeof(double2) * nb, cudaMemcpyHostToDevice) != cudaSuccess ||
-        cudaMemcpy(c->d_offsets, offsets, sizeof(int64_t) * n_offsets, cudaMemcpyHostToDevice) != cudaSuccess) {
+        cudaMemcpy(c->d_offsets, offsets, sizeof(int64_t) * n_offsets, cudaMemcpyHostToDevice) != cudaSuccess ||
+        cudaMemset(c->d_zero_offset, 0, sizeof(int64_t)) != cudaSuccess) {
         free_stats(c);
         return TRI_ECUDA;
     }
@@ -998,6 +1161,11 @@ tri_status tri_prune_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int
 tri_status tri_score(tri_ctx *c, const tri_kv *kv, const int32_t *t, float *raw, float *zmax, void *stream) {
     NvtxRange r("tri_score");
     return run(c, kv, t, 0, raw, zmax, tri::kModeScore, stream);
+}
+
+tri_status tri_decode_attention(tri_ctx *c, const tri_kv *kv, const void *q, float *out, void *stream) {
+    NvtxRange r("tri_decode_attention");
+    return run_attend(c, kv, q, out, stream);
 }
 
 tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T, int n_q_heads, int head_dim,
@@ -1063,13 +1231,9 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     if ((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps > 0x7fffffffLL) return TRI_EUNSUPPORTED;
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
-    if (kv->batch > c->seq_bad_cap) {
-        cudaFree(c->d_seq_bad);  // synchronises the device: no call still uses the old flags
-        c->d_seq_bad = nullptr;
-        c->seq_bad_cap = 0;
-        if (cudaMalloc(&c->d_seq_bad, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ENOMEM;
-        if (cudaMemset(c->d_seq_bad, 0, sizeof(int32_t) * kv->batch) != cudaSuccess) return TRI_ECUDA;
-        c->seq_bad_cap = kv->batch;
+    {
+        const tri_status fs = ensure_flags(&c->d_append_bad, &c->append_bad_cap, kv->batch);
+        if (fs != TRI_OK) return fs;
     }
     tri::AppendArgs a;
     a.K = static_cast<uint16_t *>(kv->K);
@@ -1087,7 +1251,7 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     a.max_pages = kv->max_pages;
     a.n_pages = kv->n_pages;
     a.status = c->d_status;
-    a.seq_bad = c->d_seq_bad;
+    a.seq_bad = c->d_append_bad;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
     if (c->D == 128)
@@ -1097,7 +1261,7 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append rows");
     tri::tri_append_lens_kernel<<<(unsigned)((kv->batch + 255) / 256), 256, 0, st>>>(kv->lens, kv->lens_out,
-                                                                                       c->d_seq_bad, kv->batch);
+                                                                                       c->d_append_bad, kv->batch);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append lengths");
     return TRI_OK;
@@ -1107,6 +1271,14 @@ tri_status tri_set_offset_combine(tri_ctx *c, int combine) {
     if (!c) return TRI_EINVAL;
     if (combine != TRI_OFFSETS_MEAN && combine != TRI_OFFSETS_MAX) return TRI_EINVAL;
     c->combine = combine;
+    return TRI_OK;
+}
+
+tri_status tri_set_score_engine(tri_ctx *c, int engine) {
+    if (!c) return TRI_EINVAL;
+    if (engine != TRI_ENGINE_AUTO && engine != TRI_ENGINE_CUDA_CORES && engine != TRI_ENGINE_TENSOR)
+        return TRI_EINVAL;
+    c->engine = engine;
     return TRI_OK;
 }
 
@@ -1134,6 +1306,30 @@ tri_status tri_get_error(tri_ctx *c, void *stream, int32_t *detail_code, int64_t
     if (detail_code) *detail_code = (int32_t)(v >> 32);
     if (detail_unit) *detail_unit = (int64_t)(uint32_t)(v & 0xffffffffu);
     return TRI_EDEVICE;
+}
+
+tri_status tri_get_failed_units(tri_ctx *c, void *stream, int32_t *units, int32_t capacity, int32_t *count) {
+    if (count) *count = 0;
+    if (!c || capacity < 0 || (capacity > 0 && !units)) return TRI_EINVAL;
+    if (cudaSetDevice(c->device) != cudaSuccess) return TRI_ECUDA;
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TRI_ECUDA;
+    unsigned n = 0;
+    if (cudaMemcpy(&n, c->d_fail_count, sizeof n, cudaMemcpyDeviceToHost) != cudaSuccess) return TRI_ECUDA;
+    const int listed = (int)std::min<unsigned>(n, (unsigned)std::min(capacity, kFailCap));
+    if (listed > 0 &&
+        cudaMemcpy(units, c->d_fail_units, sizeof(int32_t) * listed, cudaMemcpyDeviceToHost) != cudaSuccess)
+        return TRI_ECUDA;
+    if (n > 0 && cudaMemset(c->d_fail_count, 0, sizeof n) != cudaSuccess) return TRI_ECUDA;
+    if (count) *count = (int32_t)std::min<unsigned>(n, 0x7fffffffu);
+    return TRI_OK;
+}
+
+tri_status tri_set_test_fault(tri_ctx *c, int64_t unit, int32_t wait_tries) {
+    if (!c) return TRI_EINVAL;
+    if (wait_tries < 0 || unit < -1) return TRI_EINVAL;
+    c->inject_unit = unit;
+    c->wait_tries = wait_tries > 0 ? wait_tries : tri::kWaitTries;
+    return TRI_OK;
 }
 
 const char *tri_last_error(tri_ctx *c) {

@@ -63,7 +63,8 @@ constexpr int kDevLenGtCap = 1;
 constexpr int kDevBadPage = 2;
 constexpr int kDevTimeout = 3;
 constexpr int kDevInternal = 4;
-constexpr int kWaitTries = 1024;             // bounded mbarrier waits ...
+constexpr int kDevTNotAfterPos = 5;
+constexpr int kWaitTries = 1024;             // bounded mbarrier waits (the default number of tries) ...
 constexpr unsigned kWaitSuspendNs = 1000000; // ... each suspending the warp for up to 1 ms
 
 struct Args {
@@ -97,6 +98,11 @@ struct Args {
     const float *pre;            // precomputed scores [n_units][cap_u][G] (max-over-offsets mode)
     const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing
     long long unit_base;         // added to the unit index in device status reports
+    int wait_tries;              // tries (about 1 ms each) of every bounded wait
+    long long inject_unit;       // test hook: the unit whose first key copy is withheld (-1: none)
+    unsigned *fail_count;        // units left uncompacted by a unit-level failure ...
+    int32_t *fail_units;         // ... and the first fail_cap of them
+    int fail_cap;
 };
 
 // Per-CTA values other CTAs of the cluster read through distributed shared memory.
@@ -199,9 +205,9 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, unsigned parity) {
     return ok != 0;
 }
 
-// Bounded wait (about one second at most): returns false if the phase never completed.
-__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity) {
-    for (int i = 0; i < kWaitTries; ++i)
+// Bounded wait (tries x about 1 ms at most): returns false if the phase never completed.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, unsigned parity, int tries) {
+    for (int i = 0; i < tries; ++i)
         if (mbar_try_wait(bar, parity)) return true;
     return false;
 }
@@ -265,6 +271,18 @@ __device__ __forceinline__ unsigned float_key(float z) {
 __device__ __forceinline__ void record_status(unsigned long long *st, int code, long long unit) {
     unsigned long long v = ((unsigned long long)(unsigned)code << 32) | (unsigned long long)(unsigned)unit;
     atomicCAS(st, 0ull, v);
+}
+
+// A unit-level failure: the unit is left uncompacted (its first min(len, B) slots keep their
+// original rows), the status word records the first problem, and the unit joins the list the
+// host reads with tri_get_failed_units.
+__device__ __forceinline__ void record_unit_failure(unsigned long long *st, unsigned *fail_count,
+                                                    int32_t *fail_units, int fail_cap, int code, long long unit) {
+    record_status(st, code, unit);
+    if (fail_count) {
+        const unsigned k = atomicAdd(fail_count, 1u);
+        if ((int)k < fail_cap) fail_units[k] = (int32_t)unit;
+    }
 }
 
 // Row index (in rows of head_dim elements) of logical slot i of a unit.
@@ -338,6 +356,57 @@ __device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 in
         __syncthreads();
     }
     return carry;
+}
+
+// ---------------------------------------------------------------------------------
+// Sequence-level checks of one call, run before any unit of the call is touched, so that
+// every unit of a sequence gets the same verdict: the length within the capacity, every page
+// of the sequence inside the pool, and every unit's last cached position below t (positions
+// ascend within a unit, so the last one is the largest). One block per sequence;
+// seq_bad[s] receives the problem code (0: accepted), which the fused kernel and the
+// max-over-offsets scoring kernel read. The first problem also goes to the status word.
+// ---------------------------------------------------------------------------------
+constexpr int kValidateThreads = 256;
+
+__global__ void __launch_bounds__(kValidateThreads) tri_validate_kernel(const Args a) {
+    const int s = blockIdx.x;
+    const int N = __ldg(a.lens + s);
+    const int n_layers = a.n_units / (a.batch * a.n_kv);
+    __shared__ int bad_unit_s;
+    if (threadIdx.x == 0) bad_unit_s = 0x7fffffff;
+    __syncthreads();
+    int code = 0;
+    long long unit = (long long)s * a.n_kv;  // the sequence's first unit of the call
+    if (N < 0 || N > a.cap_u) {
+        code = kDevLenGtCap;
+    } else if (N > 0) {  // uniform over the block
+        if (a.paged) {
+            const int np = (N + a.page_size - 1) / a.page_size;
+            int mine = 0;
+            for (int p = threadIdx.x; p < np; p += kValidateThreads) {
+                const int pg = __ldg(a.block_table + (long long)s * a.max_pages + p);
+                if (pg < 0 || pg >= a.n_pages) mine = 1;
+            }
+            if (__syncthreads_or(mine)) code = kDevBadPage;
+        }
+        if (!code && a.pos) {
+            const int tq = __ldg(a.t + s);
+            for (int k = threadIdx.x; k < n_layers * a.n_kv; k += kValidateThreads) {
+                const int lr = k / a.n_kv, g = k % a.n_kv;
+                if (__ldg(a.pos + row_of(a, lr, s, g, N - 1)) >= tq)
+                    atomicMin(&bad_unit_s, (lr * a.batch + s) * a.n_kv + g);
+            }
+            __syncthreads();
+            if (bad_unit_s != 0x7fffffff) {
+                code = kDevTNotAfterPos;
+                unit = bad_unit_s;
+            }
+        }
+    }
+    if (threadIdx.x == 0) {
+        a.seq_bad[s] = code;
+        if (code) record_status(a.status, code, a.unit_base + unit);
+    }
 }
 
 // ---------------------------------------------------------------------------------
@@ -502,6 +571,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
     const bool writer = (sub & (LPK / G - 1)) == 0;
     const int Hq = a.n_kv * G;
 
+    const int tries = a.wait_tries;
     // set once a bounded wait of this cluster ran out: the ring's barrier phases can no longer
     // be trusted, so the cluster refuses its remaining units instead of streaming them
     bool dead = false;
@@ -511,33 +581,21 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
         const int lr = unit / (a.n_kv * a.batch);
         const int layer = a.layer_begin + lr;
         const int N = __ldg(a.lens + s);
+        // sequences refused by the validation kernel (length, pages, positions against t) are
+        // skipped whole; the capacity test is repeated here so that no access depends on it
+        const bool bad = __ldg(a.seq_bad + s) != 0 || N < 0 || N > a.cap_u;
+        const bool work0 = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
         if (dead) {  // uniform over the cluster
-            if (crank == 0 && tid == 0) {
-                record_status(a.status, kDevTimeout, a.unit_base + unit);
-                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
-            }
+            if (work0 && crank == 0 && tid == 0)
+                record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
+                                    a.unit_base + unit);
             continue;
         }
-
-        // ---- validation: every CTA of the cluster reaches the same verdict ----------
-        int bad = (N < 0 || N > a.cap_u) ? kDevLenGtCap : 0;
-        if (!bad && a.paged) {
-            const int np = (N + a.page_size - 1) / a.page_size;
-            int mine = 0;
-            for (int p = tid; p < np; p += kThreads) {
-                const int pg = __ldg(a.block_table + (long long)s * a.max_pages + p);
-                if (pg < 0 || pg >= a.n_pages) mine = 1;
-            }
-            if (__syncthreads_or(mine)) bad = kDevBadPage;
-        }
-        if (bad && crank == 0 && tid == 0) {
-            record_status(a.status, bad, a.unit_base + unit);
-            if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
-        }
         bool missing = false;  // the scoring kernel gave up on this unit (it recorded why)
-        if constexpr (PRE) missing = !bad && __ldg(a.unit_fail + unit) != 0;
-        if (missing && crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
-        const bool work = !bad && !missing && N > 0 && (a.mode == kModeScore || N > a.budget);
+        if constexpr (PRE) missing = work0 && __ldg(a.unit_fail + unit) != 0;
+        if (missing && crank == 0 && tid == 0)
+            record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout, a.unit_base + unit);
+        const bool work = work0 && !missing;
         if (!work) continue;  // uniform over the cluster: no cluster barrier is skipped unevenly
 
         const int kpc = ((N + cs - 1) / cs + 31) / 32 * 32;
@@ -555,7 +613,7 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             sc_read = a.pre + ((long long)unit * a.cap_u + begin) * G;
         } else {
         // ---- start streaming this CTA's keys (TMA bulk copies, per-warp buffers) -----
-        auto issue = [&](int st) {
+        auto issue = [&](int st, bool withhold) {
             const int slot = wr_slot;
             const int row0 = st * kStageRows;
             const int nrows = min(kStageRows, n_local - row0);
@@ -563,14 +621,18 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             uint64_t *bar = bars + warp * nslot + slot;
             fence_proxy_async_smem();
             mbar_expect_tx(bar, (unsigned)nrows * D * 2u);
+            if (withhold) return;
             tma_load_1d(ring + (size_t)(warp * nslot + slot) * kStageBytes, a.K + r * D,
                         (unsigned)nrows * D * 2u, bar, pol_first);
         };
         __syncthreads();  // the ring is free (previous unit's staging reads are done)
         {
+            // test hook: the unit's first copy (stage 0: warp 0 of the cluster's first CTA) is
+            // withheld, so that the wait for it runs out
+            const bool hook = crank == 0 && warp == 0 && a.unit_base + unit == a.inject_unit;
             const int pre = min(nslot, my_stages);
             for (int k = 0; k < pre; ++k) {
-                if (lane == 0) issue(warp + k * kWarps);
+                if (lane == 0) issue(warp + k * kWarps, hook && k == 0);
                 if (++wr_slot == nslot) wr_slot = 0;
             }
         }
@@ -626,14 +688,14 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
         for (int k = 0; k < my_stages; ++k) {
             const int st = warp + k * kWarps;
             const int slot = rd_slot;
-            const bool landed = __all_sync(FULL, mbar_wait_bounded(bars + warp * nslot + slot, rd_phase));
+            const bool landed = __all_sync(FULL, mbar_wait_bounded(bars + warp * nslot + slot, rd_phase, tries));
             if (!landed) {
                 // give the copies this warp still has in flight a bounded chance to land
                 int sl = slot;
                 unsigned ph = rd_phase;
                 for (int j = k + 1; j < min(my_stages, k + nslot); ++j) {
                     if (++sl == nslot) { sl = 0; ph ^= 1u; }
-                    (void)mbar_wait_bounded(bars + warp * nslot + sl, ph);
+                    (void)mbar_wait_bounded(bars + warp * nslot + sl, ph, tries);
                 }
                 fail = 1;
                 break;
@@ -710,18 +772,12 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             __syncwarp();
             if (++rd_slot == nslot) { rd_slot = 0; rd_phase ^= 1u; }
             if (k + nslot < my_stages) {
-                if (lane == 0) issue(warp + (k + nslot) * kWarps);
+                if (lane == 0) issue(warp + (k + nslot) * kWarps, false);
                 if (++wr_slot == nslot) wr_slot = 0;
             }
         }
         }  // !PRE
-        if (__syncthreads_or(fail)) {
-            if (tid == 0) {
-                record_status(a.status, kDevTimeout, a.unit_base + unit);
-                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
-            }
-            fail = 1;
-        }
+        if (__syncthreads_or(fail)) fail = 1;
 
         // ---- per-head moments over the whole unit (fp64, cluster-wide) ---------------------
         // Lanes that hold the same head differ only in their key-group bits: fold those in
@@ -838,6 +894,9 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             int f = 0;
             for (int c = 0; c < cs; ++c) f |= part_fail[c];
             anyfail_s = f;
+            if (f && crank == 0)
+                record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
+                                    a.unit_base + unit);
         }
         __syncthreads();
         dead = anyfail_s != 0;
@@ -1029,10 +1088,9 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
             // the mask must hold exactly M keys; anything else is an internal error and the
             // unit is left untouched rather than copied from a wrong index
             const bool count_ok = total == M;
-            if (!count_ok && crank == 0 && tid == 0) {
-                record_status(a.status, kDevInternal, a.unit_base + unit);
-                if (a.seq_bad) atomicExch(a.seq_bad + s, 1);
-            }
+            if (!count_ok && crank == 0 && tid == 0)
+                record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevInternal,
+                                    a.unit_base + unit);
 
             // ---- in-place stable compaction ------------------------------------------------
             // Kept rows never move to a higher slot. The only sources a write to [0, M) can
@@ -1121,8 +1179,6 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
                 }
                 __syncthreads();
             }
-        } else if (a.mode == kModePrune && anyfail_s) {
-            if (crank == 0 && tid == 0 && a.seq_bad) atomicExch(a.seq_bad + s, 1);
         }
         // the next unit reuses this CTA's exchange buffers and masks: nobody may still be
         // reading them
@@ -1141,10 +1197,12 @@ __global__ void __launch_bounds__(cta_threads(G), kMinBlocks) tri_fused_kernel(c
         __syncthreads();
         if (last_s) {
             __threadfence();
+            // a sequence refused by the validation kernel keeps its length; every other one
+            // gets min(len, B), including one with a unit left uncompacted by a unit-level
+            // failure (that unit then holds its first min(len, B) original rows)
             for (int q = tid; q < a.batch; q += kThreads) {
                 const int n = a.lens[q];
-                const int refused = a.seq_bad ? atomicExch(a.seq_bad + q, 0) : 0;
-                a.lens_out[q] = refused ? n : min(n, a.budget);
+                a.lens_out[q] = a.seq_bad[q] ? n : min(n, a.budget);
             }
             __syncthreads();
             if (tid == 0) atomicExch(a.counter, 0u);

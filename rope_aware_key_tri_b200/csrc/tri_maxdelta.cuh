@@ -23,16 +23,22 @@
 //             about 16 significant bits of C while the key stays exact.
 //   MMA       per 128-key tile: d/16 k-steps, each an M=128, N=NCOL, K=16 MMA for hi and one
 //             for lo, both accumulating into the same fp32 TMEM accumulator.
-//   epilogue  4 warps, one TMEM lane (key) per thread: the max over each head's |D|
-//             columns, plus the norm score from the key row still in shared memory; the
-//             scores go to a [unit][slot][G] fp32 buffer that the fused kernel's z-score,
-//             select and compaction read instead of scoring the keys themselves.
+//   epilogue  two warpgroups of 4 warps take the tiles in turn, one TMEM lane (key) per
+//             thread: the max over each head's columns (a head owns NOFF consecutive columns,
+//             NOFF a compile-time count, the last offset repeated when the set is smaller,
+//             so the max unrolls into three-input max instructions), plus the norm score from
+//             the key row still in shared memory (packed fp32x2 FMAs); the scores go to a
+//             [unit][slot][G] fp32 buffer that the fused kernel's z-score, select and
+//             compaction read instead of scoring the keys themselves.
 //
 // One CTA per SM, warp-specialised: warp 0 issues the TMA loads, warp 1 owns the TMEM
-// allocation and issues the MMAs, warps 2-5 run the epilogue. Key tiles stream through a
-// ring of NST stages; accumulators are double-buffered in TMEM; the coefficient image is
-// double-buffered in shared memory and reloaded only when the CTA's tile range enters a new
-// unit. Every wait is bounded; a wait that runs out records a device status, marks every unit
+// allocation and issues the MMAs, warps 2-9 run the epilogue. Key tiles stream through a
+// ring of NST stages; up to four accumulators live in TMEM (tile k in buffer k mod NACC, its
+// epilogue in warpgroup k mod 2); the coefficient image is double-buffered in shared memory
+// and reloaded only when the CTA's tile range enters a new unit.
+//
+// The same kernel scores the mean over the offsets on the tensor cores (NOFF = 1): the
+// coefficient of a head is then qbar A_f e^{i omega_f t}, the offset average folded in. Every wait is bounded; a wait that runs out records a device status, marks every unit
 // of the CTA's tile range so that the fused kernel leaves them untouched, and ends the CTA's
 // work.
 #pragma once
@@ -46,18 +52,25 @@
 
 namespace tri {
 
-constexpr int kMxThreads = 192;    // warp 0: TMA, warp 1: MMA + TMEM, warps 2-5: epilogue
+constexpr int kMxEpiGroups = 2;                         // epilogue warpgroups (tiles in turn)
+constexpr int kMxThreads = 64 + 128 * kMxEpiGroups;     // warp 0: TMA, warp 1: MMA + TMEM, then the epilogue
 constexpr int kMxTile = 128;       // keys per tile (the MMA's M)
 constexpr int kMxMaxStages = 6;
 constexpr unsigned kMxChunkBytes = kMxTile * 128u;  // one 64-dim chunk of a tile: 128 rows x 128 B
 
-// Columns of the coefficient matrix: G |D| rounded up to a multiple of 16 (M = 128 needs
+// Columns per head: the offset count padded to one of three compile-time counts (the padding
+// repeats the last offset, which leaves the maximum unchanged).
+__host__ __device__ constexpr int mx_noff_pad(int n_off) { return n_off <= 1 ? 1 : n_off <= 17 ? 17 : 32; }
+// Columns of the coefficient matrix: G NOFF rounded up to a multiple of 16 (M = 128 needs
 // N % 16 == 0, 16 <= N <= 256).
-__host__ __device__ constexpr int mx_ncol(int G, int n_off) { return (G * n_off + 15) / 16 * 16; }
+__host__ __device__ constexpr int mx_ncol(int G, int noff) { return (G * noff + 15) / 16 * 16; }
 // TMEM columns per accumulator buffer (a power of two, at least 32).
 __host__ __device__ constexpr int mx_acc_cols(int ncol) {
     return ncol <= 32 ? 32 : ncol <= 64 ? 64 : ncol <= 128 ? 128 : 256;
 }
+// Accumulator buffers: as many as 512 TMEM columns hold, at most 4 (a multiple of the
+// epilogue warpgroups, so that one warpgroup owns every tile of a buffer).
+__host__ __device__ constexpr int mx_nacc(int acc_cols) { return 512 / acc_cols < 4 ? 512 / acc_cols : 4; }
 // Bytes of one half (hi or lo) of a coefficient image: d/64 chunks of NCOL rows x 128 B.
 __host__ __device__ constexpr unsigned mx_half_bytes(int D, int ncol) { return (unsigned)(D / 64) * ncol * 128u; }
 // Whole image: hi, lo, then the norm weights [G][F] fp32; a multiple of 1024 bytes.
@@ -74,8 +87,8 @@ struct MxArgs {
     int layer_begin, n_layers;
     int min_len;                 // units with N <= min_len need no scores (prune: the budget)
     int n_off;                   // offsets per head
+    int noffp;                   // columns per head (n_off padded)
     int ncol;                    // MMA N
-    int acc_cols;                // TMEM columns per accumulator buffer
     int nst;                     // key-tile stages
     int piece_rows;              // rows per TMA box (divides 128 and the page size)
     const double2 *qbar;         // [L][Hq][F] pre-RoPE query centres (complex)
@@ -89,6 +102,9 @@ struct MxArgs {
     int32_t *unit_fail;          // [n_units]
     unsigned long long *status;
     long long unit_base;         // added to the unit index in device status reports
+    const int32_t *seq_bad;      // [batch] sequences refused by the validation kernel (no tiles)
+    int wait_tries;              // tries (about 1 ms each) of every bounded wait
+    long long inject_unit;       // test hook: the unit whose first key tile is withheld (-1: none)
 };
 
 // ---------------------------------------------------------------------------------
@@ -136,8 +152,9 @@ __device__ __forceinline__ void mx_commit(uint64_t *bar) {
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
-    uint32_t r[16];
+// 16 accumulator columns of this warp's 32 TMEM lanes, without waiting: the registers are valid
+// after tmem_wait_ld (which takes them as operands, so no use can move above the wait).
+__device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
         "%14, %15}, [%16];"
@@ -145,9 +162,31 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr)
         : "memory");
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+// Orders later uses of r after a tcgen05.wait::ld issued just before (no instruction).
+__device__ __forceinline__ void tmem_after_wait(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15])
+                 :
+                 : "memory");
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
 }
 
 // ---------------------------------------------------------------------------------
@@ -157,8 +196,8 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16]) {
 // ---------------------------------------------------------------------------------
 struct MxWalk {
     int lr, s, g, tile, tps, N;
-    __device__ __forceinline__ static int tiles_of(const MxArgs &a, int n) {
-        return (n > a.min_len && n <= a.cap_u) ? (n + kMxTile - 1) / kMxTile : 0;
+    __device__ __forceinline__ static int tiles_of(const MxArgs &a, int s, int n) {
+        return (n > a.min_len && n <= a.cap_u && __ldg(a.seq_bad + s) == 0) ? (n + kMxTile - 1) / kMxTile : 0;
     }
     __device__ __forceinline__ void start(const MxArgs &a, long long T, int per_layer) {
         lr = (int)(T / per_layer);
@@ -170,7 +209,7 @@ struct MxWalk {
         }
         s = lo;
         N = __ldg(a.lens + s);
-        tps = tiles_of(a, N);
+        tps = tiles_of(a, s, N);
         const int y = x - __ldg(a.tile_prefix + s);
         g = y / tps;
         tile = y % tps;
@@ -186,7 +225,7 @@ struct MxWalk {
                 ++lr;
             }
             N = __ldg(a.lens + s);
-            tps = tiles_of(a, N);
+            tps = tiles_of(a, s, N);
         } while (tps == 0);
     }
     __device__ __forceinline__ int unit(const MxArgs &a) const { return (lr * a.batch + s) * a.n_kv + g; }
@@ -199,7 +238,7 @@ __global__ void tri_mx_prefix_kernel(const MxArgs a) {
     int run = 0;
     for (int s = 0; s < a.batch; ++s) {
         a.tile_prefix[s] = run;
-        run += a.n_kv * MxWalk::tiles_of(a, __ldg(a.lens + s));
+        run += a.n_kv * MxWalk::tiles_of(a, s, __ldg(a.lens + s));
     }
     a.tile_prefix[a.batch] = run;
 }
@@ -245,8 +284,8 @@ __global__ void __launch_bounds__(256) tri_mx_image_kernel(const MxArgs a) {
     for (int idx = threadIdx.x; idx < ncol * F; idx += blockDim.x) {
         const int n = idx / F, f = idx % F;
         double re = 0.0, im = 0.0;
-        if (n < G * a.n_off) {
-            const int h = n / a.n_off, j = n % a.n_off;
+        if (n < G * a.noffp) {
+            const int h = n / a.noffp, j = min(n % a.noffp, a.n_off - 1);
             const double2 q = a.qbar[((size_t)layer * Hq + (size_t)g * G + h) * F + f];
             const double2 e = a.phase[((size_t)s * a.n_off + j) * F + f];
             re = q.x * e.x - q.y * e.y;
@@ -282,36 +321,41 @@ __host__ __device__ inline MxLayout mx_layout(int D, int G, int ncol, int nst) {
     L.stage = 0;
     L.image = (unsigned)nst * stage_bytes;
     L.bars = L.image + 2u * mx_image_bytes(D, G, ncol);
-    // full[nst], empty[nst], bfull[2], bempty[2], accfull[2], accempty[2], TMEM address, abort flag
-    L.total = L.bars + (unsigned)(2 * nst + 8) * 8u + 16u + 1024u;  // + alignment slack
+    // full[nst], empty[nst], bfull[2], bempty[2], accfull[4], accempty[4], TMEM address, abort flag
+    L.total = L.bars + (unsigned)(2 * nst + 12) * 8u + 16u + 1024u;  // + alignment slack
     return L;
 }
 
 // ---------------------------------------------------------------------------------
-// The scoring kernel.
+// The scoring kernel. NOFF: columns per head (mx_noff_pad of the offset count).
 // ---------------------------------------------------------------------------------
-template <int D, int G, int LAYOUT>
+template <int D, int G, int LAYOUT, int NOFF>
 __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                      const MxArgs a) {
     constexpr int F = D / 2;
     constexpr int KCH = D / 64;         // 64-dim chunks (128-byte rows)
     constexpr int KSTEPS = D / 16;      // MMA k-steps per tile
+    constexpr int NCOL = mx_ncol(G, NOFF);
+    constexpr int ACC = mx_acc_cols(NCOL);
+    constexpr int NACC = mx_nacc(ACC);
+    constexpr int NE = kMxEpiGroups;
+    constexpr int REAL = G * NOFF;      // columns that hold a (head, offset) score
+    static_assert(NACC % NE == 0 && NACC * ACC <= 512, "accumulator buffers");
     constexpr unsigned kStageBytes = KCH * kMxChunkBytes;
     extern __shared__ unsigned char mx_smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(mx_smem_raw) + 1023) &
                                                             ~uintptr_t(1023));
     const int nst = a.nst;
-    const int ncol = a.ncol;
-    const MxLayout Ly = mx_layout(D, G, ncol, nst);
-    const unsigned img_bytes = mx_image_bytes(D, G, ncol);
-    const unsigned half = mx_half_bytes(D, ncol);
+    const MxLayout Ly = mx_layout(D, G, NCOL, nst);
+    const unsigned img_bytes = mx_image_bytes(D, G, NCOL);
+    const unsigned half = mx_half_bytes(D, NCOL);
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + Ly.bars);
     uint64_t *empty = full + nst;
     uint64_t *bfull = empty + nst;
     uint64_t *bempty = bfull + 2;
     uint64_t *accfull = bempty + 2;
-    uint64_t *accempty = accfull + 2;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + 2);
+    uint64_t *accempty = accfull + 4;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + 4);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -327,21 +371,23 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     if (tid == 0) {
         for (int i = 0; i < nst; ++i) {
             mbar_init(full + i, 1);
-            mbar_init(empty + i, 4);
+            mbar_init(empty + i, 4);  // the 4 warps of the warpgroup that took the tile
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(bfull + i, 1);
-            mbar_init(bempty + i, 1 + 4);  // the MMA warp's commit and the 4 epilogue warps
+            mbar_init(bempty + i, 1 + 4 * NE);  // the MMA warp's commit and every epilogue warp
+        }
+        for (int i = 0; i < NACC; ++i) {
             mbar_init(accfull + i, 1);
             mbar_init(accempty + i, 4);
         }
         *abort_flag = 0;
         mbar_init_fence();
     }
-    const unsigned tmem_cols = (unsigned)(2 * a.acc_cols) < 32u ? 32u : (unsigned)(2 * a.acc_cols);
+    constexpr unsigned kTmemCols = (unsigned)(NACC * ACC) < 32u ? 32u : (unsigned)(NACC * ACC);
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
-                     "r"(tmem_cols)
+                     "r"(kTmemCols)
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
@@ -380,7 +426,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 if (*abort_flag) break;
                 const int unit = wk.unit(a);
                 const int stage = k % nst;
-                if (k >= nst && !mbar_wait_bounded(empty + stage, (unsigned)((k / nst - 1) & 1))) {
+                if (k >= nst && !mbar_wait_bounded(empty + stage, (unsigned)((k / nst - 1) & 1), a.wait_tries)) {
                     fail(unit);
                     break;
                 }
@@ -388,7 +434,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                     ++seg;
                     prev_unit = unit;
                     const int ub = seg & 1;
-                    if (seg >= 2 && !mbar_wait_bounded(bempty + ub, (unsigned)((seg / 2 - 1) & 1))) {
+                    if (seg >= 2 && !mbar_wait_bounded(bempty + ub, (unsigned)((seg / 2 - 1) & 1), a.wait_tries)) {
                         fail(unit);
                         break;
                     }
@@ -414,7 +460,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 fence_proxy_async_smem();
                 mbar_expect_tx(full + stage, bytes);
                 unsigned char *dst = smem + Ly.stage + (unsigned)stage * kStageBytes;
-                for (int p = 0; p < n_pieces; ++p) {
+                // test hook: the unit's first tile is armed but never loaded, so its wait runs out
+                const bool withhold = wk.tile == 0 && a.unit_base + unit == a.inject_unit;
+                for (int p = 0; p < (withhold ? 0 : n_pieces); ++p) {
                     const int r0 = wk.tile * kMxTile + p * pr;
                     if (r0 >= wk.N) break;
                     long long row;
@@ -436,15 +484,15 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
             }
             // copies still in flight must land before the CTA exits
             for (int k = (issued > nst ? issued - nst : 0); k < issued; ++k)
-                (void)mbar_wait_bounded(full + k % nst, (unsigned)((k / nst) & 1));
+                (void)mbar_wait_bounded(full + k % nst, (unsigned)((k / nst) & 1), a.wait_tries);
             for (int sg = (seg > 1 ? seg - 1 : 0); sg <= seg; ++sg)
-                (void)mbar_wait_bounded(bfull + (sg & 1), (unsigned)((sg / 2) & 1));
+                (void)mbar_wait_bounded(bfull + (sg & 1), (unsigned)((sg / 2) & 1), a.wait_tries);
         }
         __syncwarp();
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc = mx_idesc(ncol);
+            const uint32_t idesc = mx_idesc(NCOL);
             MxWalk wk;
             wk.start(a, T0, per_layer);
             int seg = -1, prev_unit = -1;
@@ -456,30 +504,30 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 if (unit != prev_unit) {
                     ++seg;
                     prev_unit = unit;
-                    if (!mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1))) {
+                    if (!mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1), a.wait_tries)) {
                         fail(unit);
                         break;
                     }
                 }
-                const int ab = k & 1;
-                if (k >= 2 && !mbar_wait_bounded(accempty + ab, (unsigned)((k / 2 - 1) & 1))) {
+                const int ab = k % NACC;
+                if (k >= NACC && !mbar_wait_bounded(accempty + ab, (unsigned)((k / NACC - 1) & 1), a.wait_tries)) {
                     fail(unit);
                     break;
                 }
-                if (!mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1))) {
+                if (!mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1), a.wait_tries)) {
                     fail(unit);
                     break;
                 }
                 tc_fence_after();
                 const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
                 const unsigned char *Bs = smem + Ly.image + (seg & 1) * img_bytes;
-                const uint32_t dt = tmem_base + (uint32_t)(ab * a.acc_cols);
+                const uint32_t dt = tmem_base + (uint32_t)(ab * ACC);
 #pragma unroll
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const unsigned koff = (unsigned)(ks & 3) * 32u;  // K = 16 bf16 = 32 bytes per step
                     const uint64_t ad = mx_desc(As + (ks >> 2) * kMxChunkBytes + koff);
-                    const uint64_t bh = mx_desc(Bs + (unsigned)(ks >> 2) * ncol * 128u + koff);
-                    const uint64_t bl = mx_desc(Bs + half + (unsigned)(ks >> 2) * ncol * 128u + koff);
+                    const uint64_t bh = mx_desc(Bs + (unsigned)(ks >> 2) * NCOL * 128u + koff);
+                    const uint64_t bl = mx_desc(Bs + half + (unsigned)(ks >> 2) * NCOL * 128u + koff);
                     mx_mma(dt, ad, bh, idesc, ks > 0 ? 1 : 0);
                     mx_mma(dt, ad, bl, idesc, 1);
                 }
@@ -490,138 +538,162 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
             }
             // every MMA issued must have completed before the TMEM is released
             if (issued > 0)
-                (void)mbar_wait_bounded(accfull + ((issued - 1) & 1), (unsigned)(((issued - 1) / 2) & 1));
+                (void)mbar_wait_bounded(accfull + (issued - 1) % NACC, (unsigned)(((issued - 1) / NACC) & 1),
+                                        a.wait_tries);
         }
         __syncwarp();
     } else {
-        // ---------------- epilogue: warps 2-5, TMEM lanes 32 * (warp % 4) ... ----------------
-        const int q = warp & 3;
+        // ---------------- epilogue: warpgroup wg takes tiles k = wg (mod NE) ----------------
+        const int ew = warp - 2;
+        const int wg = ew >> 2;
+        const int q = warp & 3;       // TMEM lane quarter this warp may access
         const int r = q * 32 + lane;  // key row within the tile
         const uint32_t lane_base = (uint32_t)(q * 32) << 16;
+        const unsigned rowoff = (unsigned)(r >> 3) * 1024u + (unsigned)(r & 7) * 128u;
         MxWalk wk;
         wk.start(a, T0, per_layer);
         int seg = -1, prev_unit = -1;
         for (int k = 0; k < count; ++k) {
             if (*abort_flag) break;
             const int unit = wk.unit(a);
-            const int stage = k % nst;
-            const int ab = k & 1;
             if (unit != prev_unit) {
                 ++seg;
                 prev_unit = unit;
             }
-            const bool ok_acc = __all_sync(0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / 2) & 1)));
-            if (!ok_acc) {
-                if (lane == 0) fail(unit);
-                break;
-            }
-            tc_fence_after();
-            // max over each head's offsets, |D| columns per head in order
-            float best[G];
+            const bool seg_end = k + 1 == count || wk.last_of_unit();
+            if (k % NE == wg) {
+                const int stage = k % nst;
+                const int ab = k % NACC;
+                const bool ok_acc =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
+                if (!ok_acc) {
+                    if (lane == 0) fail(unit);
+                    break;
+                }
+                tc_fence_after();
+                // max over each head's NOFF columns: 32 columns per wait
+                float best[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) best[h] = -__int_as_float(0x7f800000);
-            {
-                int h = 0, j = 0;
-                float cur = -__int_as_float(0x7f800000);
-                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * a.acc_cols);
-                for (int c0 = 0; c0 < ncol; c0 += 16) {
-                    float v[16];
-                    tmem_ld16(tbase + (uint32_t)c0, v);
+                for (int h = 0; h < G; ++h) best[h] = __int_as_float(0xff800000);
+                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * ACC);
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        cur = fmaxf(cur, v[i]);
-                        if (++j == a.n_off) {
+                for (int c0 = 0; c0 < REAL; c0 += 32) {
+                    uint32_t v0[16], v1[16];
+                    tmem_ld16_issue(tbase + (uint32_t)c0, v0);
+                    if (c0 + 16 < REAL) tmem_ld16_issue(tbase + (uint32_t)(c0 + 16), v1);
+                    tmem_wait_ld(v0);
+                    if (c0 + 16 < REAL) tmem_after_wait(v1);
+                    // columns pair up within a head (offsets 2j, 2j + 1) for one three-input max;
+                    // every index below is a compile-time constant once the loops unroll
 #pragma unroll
-                            for (int hh = 0; hh < G; ++hh)
-                                if (hh == h) best[hh] = cur;
-                            ++h;
-                            j = 0;
-                            cur = -__int_as_float(0x7f800000);
+                    for (int i = 0; i < 32; ++i) {
+                        const int col = c0 + i;
+                        if (col < REAL) {
+                            const int h = col / NOFF, j = col - h * NOFF;
+                            const float x = __uint_as_float(i < 16 ? v0[i] : v1[i - 16]);
+                            const bool first = (j % 2 == 0) && j + 1 < NOFF && i + 1 < 32 && col + 1 < REAL;
+                            const bool second = (j % 2 == 1) && i > 0;
+                            if (first) {
+                                const float y = __uint_as_float(i + 1 < 16 ? v0[i + 1] : v1[i + 1 - 16]);
+                                best[h] = max3f(best[h], x, y);
+                            } else if (!second) {
+                                best[h] = fmaxf(best[h], x);
+                            }
                         }
                     }
                 }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(accempty + ab);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(accempty + ab);
 
-            // norm score from the key row in the stage (the stage's TMA phase is complete:
-            // the MMA that read it has finished)
-            const bool ok_st = __all_sync(0xffffffffu, mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1)));
-            const bool ok_b = __all_sync(0xffffffffu, mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1)));
-            if (!ok_st || !ok_b) {
-                if (lane == 0) fail(unit);
-                break;
-            }
-            const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
-            const float *wsm = reinterpret_cast<const float *>(smem + Ly.image + (seg & 1) * img_bytes + 2u * half);
-            const unsigned rowoff = (unsigned)(r >> 3) * 1024u + (unsigned)(r & 7) * 128u;
-            auto piece = [&](int dim) {  // 8 dims starting at dim (a multiple of 8)
-                const unsigned off = (unsigned)(dim >> 6) * kMxChunkBytes + rowoff +
-                                     ((((unsigned)(dim & 63) >> 3) ^ (unsigned)(r & 7)) << 4);
-                return *reinterpret_cast<const uint4 *>(As + off);
-            };
-            float nrm[G];
+                // norm score from the key row in the stage (the stage's TMA phase is complete:
+                // the MMA that read it has finished)
+                const bool ok_st =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1), a.wait_tries));
+                const bool ok_b = __all_sync(
+                    0xffffffffu, mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1), a.wait_tries));
+                if (!ok_st || !ok_b) {
+                    if (lane == 0) fail(unit);
+                    break;
+                }
+                const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
+                const float *wsm =
+                    reinterpret_cast<const float *>(smem + Ly.image + (seg & 1) * img_bytes + 2u * half);
+                auto piece = [&](int dim) {  // 8 dims starting at dim (a multiple of 8)
+                    const unsigned off = (unsigned)(dim >> 6) * kMxChunkBytes + rowoff +
+                                         ((((unsigned)(dim & 63) >> 3) ^ (unsigned)(r & 7)) << 4);
+                    return *reinterpret_cast<const uint4 *>(As + off);
+                };
+                float2 nrm[G];
 #pragma unroll
-            for (int h = 0; h < G; ++h) nrm[h] = 0.f;
+                for (int h = 0; h < G; ++h) nrm[h] = make_float2(0.f, 0.f);
 #pragma unroll 2
-            for (int f0 = 0; f0 < F; f0 += 8) {
-                float nb[8];
-                if (LAYOUT == 0) {
-                    const uint4 xr = piece(f0), xi = piece(F + f0);
-                    const unsigned wr[4] = {xr.x, xr.y, xr.z, xr.w}, wi[4] = {xi.x, xi.y, xi.z, xi.w};
+                for (int f0 = 0; f0 < F; f0 += 8) {
+                    // band moduli of bands f0 .. f0 + 7, as four pairs (f, f + 1)
+                    float2 nb[4];
+                    if (LAYOUT == 0) {
+                        const uint4 xr = piece(f0), xi = piece(F + f0);
+                        const unsigned wr[4] = {xr.x, xr.y, xr.z, xr.w}, wi[4] = {xi.x, xi.y, xi.z, xi.w};
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const float r0 = bf16lo(wr[e]), r1 = bf16hi(wr[e]);
-                        const float i0 = bf16lo(wi[e]), i1 = bf16hi(wi[e]);
-                        nb[2 * e] = sqrt_approx(fmaf(r0, r0, i0 * i0));
-                        nb[2 * e + 1] = sqrt_approx(fmaf(r1, r1, i1 * i1));
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 re = make_float2(bf16lo(wr[e]), bf16hi(wr[e]));
+                            const float2 im = make_float2(bf16lo(wi[e]), bf16hi(wi[e]));
+                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
+                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
+                        }
+                    } else {
+                        const uint4 x0 = piece(2 * f0), x1 = piece(2 * f0 + 8);
+                        const unsigned wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 re = make_float2(bf16lo(wv[2 * e]), bf16lo(wv[2 * e + 1]));
+                            const float2 im = make_float2(bf16hi(wv[2 * e]), bf16hi(wv[2 * e + 1]));
+                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
+                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
+                        }
                     }
-                } else {
-                    const uint4 x0 = piece(2 * f0), x1 = piece(2 * f0 + 8);
-                    const unsigned wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const float re = bf16lo(wv[e]), im = bf16hi(wv[e]);
-                        nb[e] = sqrt_approx(fmaf(re, re, im * im));
+                    for (int h = 0; h < G; ++h) {
+                        const float4 w0 = *reinterpret_cast<const float4 *>(wsm + h * F + f0);
+                        const float4 w1 = *reinterpret_cast<const float4 *>(wsm + h * F + f0 + 4);
+                        nrm[h] = __ffma2_rn(make_float2(w0.x, w0.y), nb[0], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w0.z, w0.w), nb[1], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w1.x, w1.y), nb[2], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w1.z, w1.w), nb[3], nrm[h]);
                     }
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(empty + stage);
+                const int key = wk.tile * kMxTile + r;
+                if (key < wk.N) {
+                    float sv[G];
 #pragma unroll
-                for (int h = 0; h < G; ++h) {
-                    const float4 w0 = *reinterpret_cast<const float4 *>(wsm + h * F + f0);
-                    const float4 w1 = *reinterpret_cast<const float4 *>(wsm + h * F + f0 + 4);
-                    float acc = nrm[h];
-                    acc = fmaf(w0.x, nb[0], acc);
-                    acc = fmaf(w0.y, nb[1], acc);
-                    acc = fmaf(w0.z, nb[2], acc);
-                    acc = fmaf(w0.w, nb[3], acc);
-                    acc = fmaf(w1.x, nb[4], acc);
-                    acc = fmaf(w1.y, nb[5], acc);
-                    acc = fmaf(w1.z, nb[6], acc);
-                    acc = fmaf(w1.w, nb[7], acc);
-                    nrm[h] = acc;
+                    for (int h = 0; h < G; ++h) sv[h] = best[h] + (nrm[h].x + nrm[h].y);
+                    float *dst = a.pre + ((long long)unit * a.cap_u + key) * G;
+                    if constexpr (G >= 4) {
+#pragma unroll
+                        for (int h4 = 0; h4 < G; h4 += 4)
+                            *reinterpret_cast<float4 *>(dst + h4) =
+                                make_float4(sv[h4], sv[h4 + 1], sv[h4 + 2], sv[h4 + 3]);
+                    } else if constexpr (G == 2) {
+                        *reinterpret_cast<float2 *>(dst) = make_float2(sv[0], sv[1]);
+                    } else {
+                        dst[0] = sv[0];
+                    }
                 }
             }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(empty + stage);
-                if (k + 1 == count || wk.last_of_unit()) mbar_arrive(bempty + (seg & 1));
-            }
-            const int key = wk.tile * kMxTile + r;
-            if (key < wk.N) {
-                float sv[G];
-#pragma unroll
-                for (int h = 0; h < G; ++h) sv[h] = best[h] + nrm[h];
-                float *dst = a.pre + ((long long)unit * a.cap_u + key) * G;
-                if constexpr (G >= 4) {
-#pragma unroll
-                    for (int h4 = 0; h4 < G; h4 += 4)
-                        *reinterpret_cast<float4 *>(dst + h4) = make_float4(sv[h4], sv[h4 + 1], sv[h4 + 2], sv[h4 + 3]);
-                } else if constexpr (G == 2) {
-                    *reinterpret_cast<float2 *>(dst) = make_float2(sv[0], sv[1]);
-                } else {
-                    dst[0] = sv[0];
+            if (seg_end) {
+                // every tile of this warp's warpgroup in the unit is done: release the unit's
+                // coefficient image (after its load completed, so that this arrival can only
+                // count toward this unit's use of the buffer)
+                const bool ok_b = __all_sync(
+                    0xffffffffu, mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1), a.wait_tries));
+                if (!ok_b) {
+                    if (lane == 0) fail(unit);
+                    break;
                 }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bempty + (seg & 1));
             }
             if (k + 1 < count) wk.next(a);
         }
@@ -631,7 +703,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(tmem_cols)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
                      : "memory");
     }
 }

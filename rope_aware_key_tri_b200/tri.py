@@ -22,7 +22,8 @@ LIB_PATH = os.path.join(_HERE, "lib", "libtri_b200.so")
 TRI_OK, TRI_EINVAL, TRI_ENOMEM, TRI_ECUDA, TRI_ESTATE, TRI_EDEVICE, TRI_EUNSUPPORTED = range(7)
 TRI_ROPE_HALF, TRI_ROPE_INTERLEAVED = 0, 1
 TRI_OFFSETS_MEAN, TRI_OFFSETS_MAX = 0, 1
-TRI_DEV_NONE, TRI_DEV_LEN_GT_CAP, TRI_DEV_BAD_PAGE, TRI_DEV_TIMEOUT, TRI_DEV_INTERNAL = range(5)
+TRI_ENGINE_AUTO, TRI_ENGINE_CUDA_CORES, TRI_ENGINE_TENSOR = 0, 1, 2
+TRI_DEV_NONE, TRI_DEV_LEN_GT_CAP, TRI_DEV_BAD_PAGE, TRI_DEV_TIMEOUT, TRI_DEV_INTERNAL, TRI_DEV_T_NOT_AFTER_POS = range(6)
 
 
 class tri_kv(ctypes.Structure):
@@ -67,14 +68,19 @@ def _load():
                                          ctypes.c_int, P, P, P, P]
     L.tri_append.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
+    L.tri_get_failed_units.argtypes = [P, P, P, I32, ctypes.POINTER(I32)]
+    L.tri_decode_attention.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P]
+    L.tri_set_test_fault.argtypes = [P, I64, I32]
     L.tri_set_tuning.argtypes = [P, ctypes.c_int, ctypes.c_int]
     L.tri_set_offset_combine.argtypes = [P, ctypes.c_int]
+    L.tri_set_score_engine.argtypes = [P, ctypes.c_int]
     L.tri_last_error.argtypes = [P]
     L.tri_last_error.restype = ctypes.c_char_p
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
     for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
                "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_set_tuning", "tri_set_offset_combine",
+               "tri_get_failed_units", "tri_set_test_fault", "tri_decode_attention", "tri_set_score_engine",
                "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
     return L
@@ -142,6 +148,10 @@ def tri_calibrate_estimate(ctx, q_ptr: int, n_layers: int, T: int, n_q_heads: in
                                        int(layout), q_mean_ptr, q_norm_mean_ptr, R_ptr, stream)
 
 
+def tri_decode_attention(ctx, kv: tri_kv, q_ptr: int, out_ptr: int, stream: int) -> int:
+    return _lib.tri_decode_attention(ctx, ctypes.byref(kv), q_ptr, out_ptr, stream)
+
+
 def tri_append(ctx, kv: tri_kv, k_new_ptr: int, v_new_ptr: int, pos_new_ptr: int, stream: int) -> int:
     return _lib.tri_append(ctx, ctypes.byref(kv), k_new_ptr, v_new_ptr, pos_new_ptr, stream)
 
@@ -151,6 +161,18 @@ def tri_get_error(ctx, stream: int):
     unit = ctypes.c_int64()
     st = _lib.tri_get_error(ctx, stream, ctypes.byref(code), ctypes.byref(unit))
     return st, code.value, unit.value
+
+
+def tri_get_failed_units(ctx, stream: int, capacity: int = 4096):
+    """(status, total count, list of unit indices) of units left uncompacted by unit-level failures."""
+    buf = (ctypes.c_int32 * max(1, capacity))()
+    n = ctypes.c_int32()
+    st = _lib.tri_get_failed_units(ctx, stream, buf, int(capacity), ctypes.byref(n))
+    return st, n.value, [buf[i] for i in range(min(n.value, capacity))]
+
+
+def tri_set_test_fault(ctx, unit: int = -1, wait_tries: int = 0) -> int:
+    return _lib.tri_set_test_fault(ctx, int(unit), int(wait_tries))
 
 
 def tri_last_error(ctx) -> str:
@@ -166,6 +188,10 @@ def tri_set_offset_combine(ctx, combine: int) -> int:
     return _lib.tri_set_offset_combine(ctx, int(combine))
 
 
+def tri_set_score_engine(ctx, engine: int) -> int:
+    return _lib.tri_set_score_engine(ctx, int(engine))
+
+
 # ---- torch-facing wrapper ----------------------------------------------------------------
 
 def _ptr(x: Optional[torch.Tensor]) -> Optional[int]:
@@ -176,6 +202,11 @@ def _stream_handle(stream) -> int:
     if stream is None:
         stream = torch.cuda.current_stream()
     return stream.cuda_stream
+
+
+def _check_t(t, lens):
+    if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous() or t.shape != lens.shape:
+        raise ValueError(f"t must be a contiguous CUDA int32 tensor shaped like lens {tuple(lens.shape)}")
 
 
 def make_kv(K, V, pos, lens, lens_out=None, block_table=None, n_pages=None, layer_begin=0) -> tri_kv:
@@ -192,6 +223,16 @@ def make_kv(K, V, pos, lens, lens_out=None, block_table=None, n_pages=None, laye
             continue
         if x.dtype != dt or not x.is_cuda or not x.is_contiguous():
             raise ValueError(f"{name} must be a contiguous CUDA tensor of {dt}")
+    # the C ABI sees plain pointers: check here that every buffer holds what the call describes
+    batch = int(lens.shape[0])
+    if K.dim() != 5 or (V is not None and V.shape != K.shape):
+        raise ValueError("K (and V) must be 5-D: [L][batch][Hkv][cap][d] dense or [L][pages][Hkv][page][d] paged")
+    if pos is not None and tuple(pos.shape) != tuple(K.shape[:4]):
+        raise ValueError(f"pos must be {tuple(K.shape[:4])}, got {tuple(pos.shape)}")
+    if block_table is None and int(K.shape[1]) != batch:
+        raise ValueError(f"dense cache holds {int(K.shape[1])} sequences, lens describes {batch}")
+    if block_table is not None and (block_table.dim() != 2 or int(block_table.shape[0]) != batch):
+        raise ValueError(f"block_table must be [batch={batch}][max_pages]")
     kv = tri_kv()
     kv.K, kv.V, kv.pos = _ptr(K), _ptr(V), _ptr(pos)
     kv.lens, kv.lens_out, kv.block_table = _ptr(lens), _ptr(lens_out), _ptr(block_table)
@@ -239,6 +280,14 @@ class TriContext:
         if st != TRI_OK:
             raise TriError(st, "tri_set_offset_combine")
 
+    def set_score_engine(self, engine):
+        """"auto" (the default), "cuda_cores" or "tensor" (or the TRI_ENGINE_* value)."""
+        code = {"auto": TRI_ENGINE_AUTO, "cuda_cores": TRI_ENGINE_CUDA_CORES, "tensor": TRI_ENGINE_TENSOR}.get(
+            engine, engine)
+        st = tri_set_score_engine(self.handle, code)
+        if st != TRI_OK:
+            raise TriError(st, "tri_set_score_engine")
+
     def set_tuning(self, cluster_size=0, buffers_per_warp=0):
         st = tri_set_tuning(self.handle, cluster_size, buffers_per_warp)
         if st != TRI_OK:
@@ -249,8 +298,7 @@ class TriContext:
         if isinstance(lens_out, str):
             lens_out = lens
         kv = make_kv(K, V, pos, lens, lens_out, block_table, layer_begin=layer_begin)
-        if t.dtype != torch.int32 or not t.is_cuda:
-            raise ValueError("t must be a CUDA int32 tensor")
+        _check_t(t, lens)
         st = tri_prune(self.handle, kv, t.data_ptr(), budget, _stream_handle(stream))
         if check and st != TRI_OK:
             raise TriError(st, "tri_prune", tri_last_error(self.handle))
@@ -262,6 +310,7 @@ class TriContext:
         if isinstance(lens_out, str):
             lens_out = lens
         kv = make_kv(K, V, pos, lens, lens_out, block_table, layer_begin=layer_begin)
+        _check_t(t, lens)
         st = tri_prune_noalloc(self.handle, kv, t.data_ptr(), budget, _stream_handle(stream))
         if check and st != TRI_OK:
             raise TriError(st, "tri_prune_noalloc", tri_last_error(self.handle))
@@ -270,6 +319,7 @@ class TriContext:
     def score(self, K, lens, t, raw=None, zmax=None, block_table=None, layer_begin=0,
               stream=None, check=True):
         kv = make_kv(K, None, None, lens, None, block_table, layer_begin=layer_begin)
+        _check_t(t, lens)
         st = tri_score(self.handle, kv, t.data_ptr(), _ptr(raw), _ptr(zmax), _stream_handle(stream))
         if check and st != TRI_OK:
             raise TriError(st, "tri_score", tri_last_error(self.handle))
@@ -291,6 +341,28 @@ class TriContext:
         if check and st != TRI_OK:
             raise TriError(st, "tri_append", tri_last_error(self.handle))
         return st
+
+    def decode_attention(self, K, V, lens, q, out=None, block_table=None, n_pages=None, layer_begin=0,
+                         stream=None, check=True):
+        """Attention of the post-RoPE queries q (bf16 [n_layers][batch][Hq][d]) over the cached
+        rows [0, lens[s]) of K/V (layouts as in make_kv). Returns out (fp32, like q), or the
+        status when check is False."""
+        kv = make_kv(K, V, None, lens, None, block_table, n_pages=n_pages, layer_begin=layer_begin)
+        if q.dtype != torch.bfloat16 or not q.is_cuda or not q.is_contiguous():
+            raise ValueError("q must be a contiguous CUDA tensor of torch.bfloat16")
+        if q.dim() != 4 or tuple(q.shape[:2]) != (int(K.shape[0]), int(lens.shape[0])) or q.shape[3] != K.shape[4]:
+            raise ValueError(f"q must be [n_layers][batch][Hq][d] for this cache, got {tuple(q.shape)}")
+        if out is not None and (out.dtype != torch.float32 or tuple(out.shape) != tuple(q.shape)
+                                or not out.is_contiguous()):
+            raise ValueError("out must be a contiguous float32 tensor shaped like q")
+        if out is None:
+            out = torch.empty(q.shape, dtype=torch.float32, device=q.device)
+        st = tri_decode_attention(self.handle, kv, q.data_ptr(), out.data_ptr(), _stream_handle(stream))
+        if not check:
+            return st
+        if st != TRI_OK:
+            raise TriError(st, "tri_decode_attention", tri_last_error(self.handle))
+        return out
 
     def calibrate_estimate(self, Q, layout, out=None, stream=None, check=True):
         """Calibration statistics from pre-RoPE queries Q (bf16 [n_layers][T][n_q_heads][head_dim],
@@ -314,3 +386,16 @@ class TriContext:
 
     def get_error(self, stream=None):
         return tri_get_error(self.handle, _stream_handle(stream))
+
+    def failed_units(self, stream=None, capacity=4096):
+        """(total count, unit indices) of units left uncompacted by unit-level failures."""
+        st, n, units = tri_get_failed_units(self.handle, _stream_handle(stream), capacity)
+        if st != TRI_OK:
+            raise TriError(st, "tri_get_failed_units")
+        return n, units
+
+    def set_test_fault(self, unit=-1, wait_tries=0):
+        """Test hook: withhold the first key copy of `unit` on later calls (-1: off)."""
+        st = tri_set_test_fault(self.handle, unit, wait_tries)
+        if st != TRI_OK:
+            raise TriError(st, "tri_set_test_fault")

@@ -19,7 +19,7 @@ SCORE_RTOL = 1e-4
 Z_TIE = 1e-4
 
 
-def context_for(cache, cluster_size=0, buffers=0, combine="mean"):
+def context_for(cache, cluster_size=0, buffers=0, combine="mean", engine="auto"):
     s = cache.spec
     ctx = tri.TriContext(0)
     ctx.calibrate_load(s.n_layers, s.n_kv_heads, s.group, s.head_dim, s.rope_base, s.layout,
@@ -28,6 +28,8 @@ def context_for(cache, cluster_size=0, buffers=0, combine="mean"):
         ctx.set_tuning(cluster_size, buffers)
     if combine != "mean":
         ctx.set_offset_combine(combine)
+    if engine != "auto":
+        ctx.set_score_engine(engine)
     return ctx
 
 
@@ -63,17 +65,43 @@ def oracle_unit(cache, u, B, rows=None, combine="mean"):
                              s.layout, combine=combine)
 
 
+def zmax_bound(s_err, s_orc, z_orc):
+    """Largest |zmax_gpu - zmax_oracle| that score errors of at most s_err[h] per head allow.
+
+    With |s_gpu - s| <= e per key, the mean moves by at most e and the population std by at
+    most 2e (the centred vectors differ by at most 2e per key), so
+    |z_gpu - z| <= (2 + 2|z|) e / (sigma - 2e); zmax, a max over the heads, moves by at most
+    the largest head bound. Added: the fp32 evaluation of (s - mu) / sigma and the max
+    (a few ulps of |z|). A flat head (sigma = 0) has z = 0 on both sides."""
+    G, n = s_orc.shape
+    bound = 0.0
+    for h in range(G):
+        sig = s_orc[h].std()
+        if not (s_orc[h].max() > s_orc[h].min()):
+            continue
+        # the kernel's mean is rounded to fp32 before the subtraction: an error of up to
+        # 2^-24 |mu| on top of the score's own
+        e = float(s_err[h]) + 2.0 ** -24 * abs(float(s_orc[h].mean()))
+        if sig <= 2 * e:
+            return np.inf
+        bound = max(bound, (2.0 + 2.0 * np.abs(z_orc[h]).max()) * e / (sig - 2 * e))
+    return bound + 4e-7 * (1.0 + np.abs(z_orc).max())
+
+
 def check_scores(raw_u, zmax_u, orc, label=""):
     """raw_u [G][n] and zmax_u [n] from the GPU against the oracle's s and zmax."""
     s = orc["s"]
     G, n = s.shape
+    errs = np.zeros(G)
     for h in range(G):
         scale = np.abs(s[h]).max() if n else 0.0
         err = np.abs(raw_u[h, :n].astype(np.float64) - s[h]).max() if n else 0.0
         assert err <= SCORE_RTOL * scale + 1e-30, f"{label} head {h}: score error {err:.3e} vs scale {scale:.3e}"
+        errs[h] = err
     if n:
         zerr = np.abs(zmax_u[:n].astype(np.float64) - orc["zmax"]).max()
-        assert zerr <= 1e-3, f"{label}: zmax error {zerr:.3e}"
+        zb = zmax_bound(errs, s, orc["z"])
+        assert zerr <= zb, f"{label}: zmax error {zerr:.3e} above the bound {zb:.3e} the score errors allow"
 
 
 def kept_from_output(in_pos, out_pos):

@@ -319,8 +319,9 @@ def pin_prune_batch_matches_units(L, seed=12):
         RR = np.stack([u[2] for u in units])
         # t differs per unit: each unit's own t (its positions all lie below it)
         tt = np.array([u[5] + 7 * i for i, u in enumerate(units)], np.int64)
-        kept, nk, zm = oracle.prune_batch(Kb, Pb, np.array(lens, np.int32), tt, qm, qn, RR, offsets, base, B,
-                                          layout, n_threads=2, want_zmax=True, L=L, combine=combine)
+        kept, nk, zm, sc = oracle.prune_batch(Kb, Pb, np.array(lens, np.int32), tt, qm, qn, RR, offsets, base, B,
+                                              layout, n_threads=2, want_zmax=True, L=L, combine=combine,
+                                              want_scores=True)
         for u, n in enumerate(lens):
             assert nk[u] == min(n, B), (d, G, combine, u, nk[u], n)
             if n == 0:
@@ -330,6 +331,7 @@ def pin_prune_batch_matches_units(L, seed=12):
                                     layout, L=L, combine=combine)
             assert np.array_equal(kept[u, :nk[u]], one["kept"]), (d, G, combine, u)
             assert np.array_equal(zm[u, :n], one["zmax"]), (d, G, combine, u)
+            assert np.array_equal(sc[u, :, :n], one["s"]), (d, G, combine, u)
 
 
 def pin_select_f32(L, seed=13):

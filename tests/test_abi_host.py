@@ -28,7 +28,7 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_score",
               "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_status_str",
-              "tri_set_offset_combine"):
+              "tri_set_offset_combine", "tri_decode_attention", "tri_get_failed_units", "tri_set_test_fault"):
         assert n in names
 
 
@@ -63,6 +63,10 @@ def test_host_validation_without_device(lib):
     unit = ctypes.c_int64(7)
     assert lib.tri_get_error(None, None, ctypes.byref(code), ctypes.byref(unit)) == tri.TRI_EINVAL
     assert code.value == 0 and unit.value == -1
+    assert tri.tri_decode_attention(None, kv, 0, 0, None) == tri.TRI_EINVAL
+    n = ctypes.c_int32(5)
+    assert lib.tri_get_failed_units(None, None, None, 0, ctypes.byref(n)) == tri.TRI_EINVAL and n.value == 0
+    assert lib.tri_set_test_fault(None, -1, 0) == tri.TRI_EINVAL
 
 
 def test_create_without_gpu_fails_cleanly(lib):

@@ -284,6 +284,9 @@ def make_cache(spec: CacheSpec, seed: int, device="cpu", lens=None, t=None,
         t_r = list(t)
     elif spec.positions == "from_zero":
         t_r = list(lens_r)
+    if len(lens_r) != spec.batch or len(t_r) != spec.batch:
+        raise ValueError(f"{spec.name}: {len(lens_r)} lengths and {len(t_r)} query positions for a batch of "
+                         f"{spec.batch}")
     maxlen = max(lens_r) if lens_r else 0
     omega = torch.as_tensor(rope_omega(d, spec.rope_base), device=device)
     wdtype = torch.float64  # keys drawn and rotated in fp64 on every device, then rounded RNE to bf16
