@@ -313,7 +313,8 @@ TRI_API tri_status tri_get_failed_units(tri_ctx *ctx, void *stream, int32_t *uni
  * Test hook for the failure path (not part of the paper's pass; off by default).
  *   unit        index (as in tri_get_error) of a unit whose first key copy the scoring kernels
  *               arm but never issue on the next calls, so that the wait for it runs out; -1 = off
- *   wait_tries  tries of every bounded wait, about 1 ms each (0 = the default 1024)
+ *   wait_tries  tries of the bounded waits, about 1 ms each (0 = the default 1024); the fused
+ *               CUDA-core kernel's key-stream wait keeps the default bound (about one second)
  * The withheld copy never lands, the wait gives up after wait_tries tries, the kernel records
  * TRI_DEV_TIMEOUT and leaves the affected units uncompacted (unit-level failure); no copy is
  * left in flight and nothing waits without bound.

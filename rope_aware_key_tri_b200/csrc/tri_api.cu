@@ -216,6 +216,9 @@ constexpr int kFailCap = 4096;
 // Live score slots should stay well inside the 126 MB L2 so that the scores written during
 // streaming are read back from L2.
 constexpr double kScoreL2Budget = 100.0 * 1024 * 1024;
+// Fixed cost of a unit in scored keys per CTA (fit to measured prune times of one Qwen3-8B
+// layer, 128 units of 2176 keys, over cluster sizes 1 to 16).
+constexpr double kUnitOverheadKeys = 700.0;
 
 std::mutex g_attr_mu;
 
@@ -238,11 +241,11 @@ cudaError_t prepare_kernel(KernelFn fn, int max_optin) {
 }
 
 // Clusters that can be resident at once for this shape (0 if it cannot launch).
-int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem) {
+int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem, bool pre) {
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)cs);
-    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
+    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G, pre));
     cfg.dynamicSmemBytes = smem;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -261,11 +264,14 @@ int resident_clusters(tri_ctx *c, KernelFn fn, int cs, size_t smem) {
 }
 
 // Pick the launch shape of the persistent grid. A cluster of cs CTAs shares one unit; the
-// grid holds as many clusters as can be resident (two CTAs per SM). cs is the smallest
-// power of two that (a) gives every resident CTA slot a unit to work on and (b) keeps the
-// live score slots (one per resident cluster) within the L2 budget; if none does both,
-// the largest cs that fits.
-tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Plan *out) {
+// grid holds as many clusters as can be resident (two CTAs per SM). Among the cluster sizes
+// whose live score slots (one per resident cluster) fit the L2 budget and whose per-CTA order
+// keys fit in shared memory, cs minimises the
+// estimated time waves(cs) * (cap_u / cs + kUnitOverheadKeys): the waves of units over the
+// resident clusters times a unit's work per CTA plus its fixed cost (prologue, cluster
+// exchanges, radix passes and compaction rounds, in key-equivalents). If none fits the budget,
+// the largest cs that can launch.
+tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Plan *out, bool pre) {
     auto &pc = c->plan_cache;
     if (pc.valid && pc.fn == (const void *)fn && pc.cap_u == cap_u && pc.n_units == n_units &&
         pc.tune_cs == c->tune_cs && pc.tune_nslot == c->tune_nslot) {
@@ -281,8 +287,13 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
     cudaError_t fe = cudaFuncGetAttributes(&fa, fn);
     if (fe != cudaSuccess) return cuda_fail(c, fe, "cudaFuncGetAttributes");
     const size_t budget = (size_t)c->max_smem_optin - fa.sharedSizeBytes;
-    const double unit_bytes = (double)cap_u * c->G * 4.0;  // scores; order keys usually stay on chip
+    // live bytes of a cluster's scratch slot: the scores (fused engine; the order keys usually
+    // stay on chip), or only the order keys when the scores come precomputed
+    const double unit_bytes = (double)cap_u * (pre ? 1 : c->G) * 4.0;
+    const int threads = tri::cta_threads(c->G, pre);
     Plan best;
+    bool best_fits = false;
+    double best_cost = 0.0;
     for (int cs = 1; cs <= tri::kMaxCluster; cs *= 2) {
         if (c->tune_cs > 0 && cs != c->tune_cs) continue;
         const long long kpc = ((long long)(cap_u + cs - 1) / cs + 31) / 32 * 32;
@@ -290,21 +301,21 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
         // buffers per warp: the deepest ring (3 at most) that still leaves room for two
         // CTAs per SM, else whatever fits one CTA
         int nslot = c->tune_nslot > 0 ? c->tune_nslot : 3;
-        tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0);
+        tri::Layout Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0, pre);
         int res = 0;
         for (; nslot >= 1; --nslot) {
-            Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0);
+            Ly = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, 0, pre);
             if (Ly.total > budget || Ly.stage_rows < 16) {
                 if (c->tune_nslot > 0) break;
                 continue;
             }
             int per_sm = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::cta_threads(c->G), Ly.total) != cudaSuccess) {
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, Ly.total) != cudaSuccess) {
                 cudaGetLastError();
                 per_sm = 0;
             }
             if (c->tune_nslot > 0 || per_sm >= tri::kMinBlocks || nslot == 1) {
-                res = per_sm >= 1 ? resident_clusters(c, fn, cs, Ly.total) : 0;
+                res = per_sm >= 1 ? resident_clusters(c, fn, cs, Ly.total, pre) : 0;
                 break;
             }
         }
@@ -312,16 +323,16 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
         // shared memory left over at this occupancy goes to the compaction's staging
         int extra = 0;
         for (int e = 64 * 1024; e >= 8 * 1024; e -= 8 * 1024) {
-            const tri::Layout Le = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, e);
+            const tri::Layout Le = tri::make_layout(c->D, c->G, nslot, (int)kpc, cs, e, pre);
             if (Le.total > budget) continue;
             int per_sm_e = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_e, fn, tri::cta_threads(c->G), Le.total) !=
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_e, fn, threads, Le.total) !=
                 cudaSuccess) {
                 cudaGetLastError();
                 continue;
             }
             int per_sm0 = 0;
-            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm0, fn, tri::cta_threads(c->G), Ly.total) !=
+            if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm0, fn, threads, Ly.total) !=
                 cudaSuccess) {
                 cudaGetLastError();
                 break;
@@ -339,10 +350,19 @@ tri_status plan_launch(tri_ctx *c, KernelFn fn, int cap_u, long long n_units, Pl
         p.kpc = (int)kpc;
         p.smem = Ly.total;
         p.n_clusters = (int)std::min<long long>(n_units, res);
-        best = p;
-        const bool fills = n_units * cs >= (long long)res * cs;  // every resident cluster has a unit
-        const bool fits_l2 = (double)p.n_clusters * unit_bytes <= kScoreL2Budget;
-        if (fills && fits_l2) break;
+        // the order keys of a CTA's share of a unit should fit in the (idle) ring, so that the
+        // radix passes run on chip; and the live score slots within the L2 budget
+        const bool keys_on_chip = (double)kpc * 4.0 <= (double)Ly.ring_bytes;
+        const bool fits_l2 = (double)p.n_clusters * unit_bytes <= kScoreL2Budget && keys_on_chip;
+        const double waves = (double)((n_units + res - 1) / res);
+        const double cost = waves * ((double)cap_u / cs + kUnitOverheadKeys);
+        if (fits_l2 && (!best_fits || cost < best_cost)) {
+            best = p;
+            best_fits = true;
+            best_cost = cost;
+        } else if (!best_fits) {
+            best = p;  // nothing fits the budget yet: the largest cluster size that launches
+        }
     }
     if (best.cs == 0) return TRI_EUNSUPPORTED;
     *out = best;
@@ -473,8 +493,9 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
     ce = prepare_kernel(fn, c->max_smem_optin);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute");
+    const bool is_pre = pre != nullptr;
     Plan plan;
-    tri_status st = plan_launch(c, fn, (int)cap_u, n_units, &plan);
+    tri_status st = plan_launch(c, fn, (int)cap_u, n_units, &plan, is_pre);
     if (st != TRI_OK) return st;
 
     const long long slot_floats = ((long long)cap_u * (c->G + 1) + 31) / 32 * 32;
@@ -508,7 +529,7 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
     cfg.gridDim = dim3((unsigned)(plan.n_clusters * plan.cs));
-    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
+    cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G, is_pre));
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[1];
@@ -833,7 +854,7 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     ce = prepare_kernel(fn, c->max_smem_optin);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute");
     Plan plan;
-    st = plan_launch(c, fn, (int)cap_u, n_units, &plan);
+    st = plan_launch(c, fn, (int)cap_u, n_units, &plan, false);
     if (st == TRI_EUNSUPPORTED) {
         std::snprintf(c->last_error, sizeof c->last_error,
                       "tri_prune_noalloc: no launch shape holds a unit capacity of %lld slots on chip", cap_u);

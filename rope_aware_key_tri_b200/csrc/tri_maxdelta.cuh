@@ -564,6 +564,63 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
             if (k % NE == wg) {
                 const int stage = k % nst;
                 const int ab = k % NACC;
+                // norm score first: it needs only the key rows, which usually land before the
+                // tile's MMAs finish, so this work overlaps them
+                const bool ok_st =
+                    __all_sync(0xffffffffu, mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1), a.wait_tries));
+                const bool ok_b = __all_sync(
+                    0xffffffffu, mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1), a.wait_tries));
+                if (!ok_st || !ok_b) {
+                    if (lane == 0) fail(unit);
+                    break;
+                }
+                const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
+                const float *wsm =
+                    reinterpret_cast<const float *>(smem + Ly.image + (seg & 1) * img_bytes + 2u * half);
+                auto piece = [&](int dim) {  // 8 dims starting at dim (a multiple of 8)
+                    const unsigned off = (unsigned)(dim >> 6) * kMxChunkBytes + rowoff +
+                                         ((((unsigned)(dim & 63) >> 3) ^ (unsigned)(r & 7)) << 4);
+                    return *reinterpret_cast<const uint4 *>(As + off);
+                };
+                float2 nrm[G];
+#pragma unroll
+                for (int h = 0; h < G; ++h) nrm[h] = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int f0 = 0; f0 < F; f0 += 8) {
+                    // band moduli of bands f0 .. f0 + 7, as four pairs (f, f + 1)
+                    float2 nb[4];
+                    if (LAYOUT == 0) {
+                        const uint4 xr = piece(f0), xi = piece(F + f0);
+                        const unsigned wr[4] = {xr.x, xr.y, xr.z, xr.w}, wi[4] = {xi.x, xi.y, xi.z, xi.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 re = make_float2(bf16lo(wr[e]), bf16hi(wr[e]));
+                            const float2 im = make_float2(bf16lo(wi[e]), bf16hi(wi[e]));
+                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
+                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
+                        }
+                    } else {
+                        const uint4 x0 = piece(2 * f0), x1 = piece(2 * f0 + 8);
+                        const unsigned wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const float2 re = make_float2(bf16lo(wv[2 * e]), bf16lo(wv[2 * e + 1]));
+                            const float2 im = make_float2(bf16hi(wv[2 * e]), bf16hi(wv[2 * e + 1]));
+                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
+                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
+                        }
+                    }
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        const float4 w0 = *reinterpret_cast<const float4 *>(wsm + h * F + f0);
+                        const float4 w1 = *reinterpret_cast<const float4 *>(wsm + h * F + f0 + 4);
+                        nrm[h] = __ffma2_rn(make_float2(w0.x, w0.y), nb[0], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w0.z, w0.w), nb[1], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w1.x, w1.y), nb[2], nrm[h]);
+                        nrm[h] = __ffma2_rn(make_float2(w1.z, w1.w), nb[3], nrm[h]);
+                    }
+                }
+
                 const bool ok_acc =
                     __all_sync(0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
                 if (!ok_acc) {
@@ -604,66 +661,11 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(accempty + ab);
-
-                // norm score from the key row in the stage (the stage's TMA phase is complete:
-                // the MMA that read it has finished)
-                const bool ok_st =
-                    __all_sync(0xffffffffu, mbar_wait_bounded(full + stage, (unsigned)((k / nst) & 1), a.wait_tries));
-                const bool ok_b = __all_sync(
-                    0xffffffffu, mbar_wait_bounded(bfull + (seg & 1), (unsigned)((seg / 2) & 1), a.wait_tries));
-                if (!ok_st || !ok_b) {
-                    if (lane == 0) fail(unit);
-                    break;
+                // the MMA has finished with the key tile and the accumulator: release both
+                if (lane == 0) {
+                    mbar_arrive(accempty + ab);
+                    mbar_arrive(empty + stage);
                 }
-                const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
-                const float *wsm =
-                    reinterpret_cast<const float *>(smem + Ly.image + (seg & 1) * img_bytes + 2u * half);
-                auto piece = [&](int dim) {  // 8 dims starting at dim (a multiple of 8)
-                    const unsigned off = (unsigned)(dim >> 6) * kMxChunkBytes + rowoff +
-                                         ((((unsigned)(dim & 63) >> 3) ^ (unsigned)(r & 7)) << 4);
-                    return *reinterpret_cast<const uint4 *>(As + off);
-                };
-                float2 nrm[G];
-#pragma unroll
-                for (int h = 0; h < G; ++h) nrm[h] = make_float2(0.f, 0.f);
-#pragma unroll 2
-                for (int f0 = 0; f0 < F; f0 += 8) {
-                    // band moduli of bands f0 .. f0 + 7, as four pairs (f, f + 1)
-                    float2 nb[4];
-                    if (LAYOUT == 0) {
-                        const uint4 xr = piece(f0), xi = piece(F + f0);
-                        const unsigned wr[4] = {xr.x, xr.y, xr.z, xr.w}, wi[4] = {xi.x, xi.y, xi.z, xi.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 re = make_float2(bf16lo(wr[e]), bf16hi(wr[e]));
-                            const float2 im = make_float2(bf16lo(wi[e]), bf16hi(wi[e]));
-                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
-                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
-                        }
-                    } else {
-                        const uint4 x0 = piece(2 * f0), x1 = piece(2 * f0 + 8);
-                        const unsigned wv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const float2 re = make_float2(bf16lo(wv[2 * e]), bf16lo(wv[2 * e + 1]));
-                            const float2 im = make_float2(bf16hi(wv[2 * e]), bf16hi(wv[2 * e + 1]));
-                            const float2 sq = __ffma2_rn(im, im, __fmul2_rn(re, re));
-                            nb[e] = make_float2(sqrt_approx(sq.x), sqrt_approx(sq.y));
-                        }
-                    }
-#pragma unroll
-                    for (int h = 0; h < G; ++h) {
-                        const float4 w0 = *reinterpret_cast<const float4 *>(wsm + h * F + f0);
-                        const float4 w1 = *reinterpret_cast<const float4 *>(wsm + h * F + f0 + 4);
-                        nrm[h] = __ffma2_rn(make_float2(w0.x, w0.y), nb[0], nrm[h]);
-                        nrm[h] = __ffma2_rn(make_float2(w0.z, w0.w), nb[1], nrm[h]);
-                        nrm[h] = __ffma2_rn(make_float2(w1.x, w1.y), nb[2], nrm[h]);
-                        nrm[h] = __ffma2_rn(make_float2(w1.z, w1.w), nb[3], nrm[h]);
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty + stage);
                 const int key = wk.tile * kMxTile + r;
                 if (key < wk.N) {
                     float sv[G];
