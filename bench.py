@@ -758,10 +758,12 @@ def run_attend(args):
     units = spec.n_layers * spec.batch * spec.n_kv_heads
     rows = sum(lens) * spec.n_layers * spec.n_kv_heads
     nbytes = rows * 2 * spec.head_dim * 2 + q.numel() * 2 + out.numel() * 4
-    # launches: validation, attention, and the chunk merge when units are split (two CTAs per SM)
+    # launches: validation, attention, and the chunk merge when units are split (three CTAs per
+    # SM up to GQA 4, two at GQA 8)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     cap_u = cache.cap
-    cpu = max(1, min(-(-4 * sms * 2 // units), -(-cap_u // 256)))
+    per_sm = 3 if spec.group <= 4 else 2
+    cpu = max(1, min(-(-4 * sms * per_sm // units), -(-cap_u // 256)))
     res = {"metric": ATT_METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
            "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 accumulate", "data": "synthetic",

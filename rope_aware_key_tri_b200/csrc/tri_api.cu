@@ -485,15 +485,20 @@ tri_status launch_validate(tri_ctx *c, const tri_kv *kv, const int32_t *t, int m
 // One launch of the fused kernel `fn` over the units of kv. pre / unit_fail: precomputed
 // scores (the PRE variant) or null; lens_out: where the last CTA publishes the new lengths
 // (null: not in this launch); seq_bad: the validation kernel's per-sequence verdicts.
+struct PreScores {  // what the tensor-core scoring kernel left for the fused kernel
+    const float *scores = nullptr;
+    const int32_t *unit_fail = nullptr;
+};
+
 tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t *t, int32_t budget, float *raw,
-                        float *zmax, int mode, long long cap_u, const float *pre, const int32_t *unit_fail,
-                        long long unit_base, int32_t *lens_out, int32_t *seq_bad, void *stream) {
+                        float *zmax, int mode, long long cap_u, const PreScores &pre, long long unit_base,
+                        int32_t *lens_out, int32_t *seq_bad, void *stream) {
     const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
     ce = prepare_kernel(fn, c->max_smem_optin);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute");
-    const bool is_pre = pre != nullptr;
+    const bool is_pre = pre.scores != nullptr;
     Plan plan;
     tri_status st = plan_launch(c, fn, (int)cap_u, n_units, &plan, is_pre);
     if (st != TRI_OK) return st;
@@ -522,8 +527,8 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     a.ring_extra = plan.extra;
     a.scratch = c->d_scratch;
     a.slot_floats = slot_floats;
-    a.pre = pre;
-    a.unit_fail = unit_fail;
+    a.pre = pre.scores;
+    a.unit_fail = pre.unit_fail;
     a.unit_base = unit_base;
 
     cudaLaunchConfig_t cfg;
@@ -644,6 +649,7 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
     if ((st = grow(c, &c->d_unit_fail, &c->unit_fail_bytes, (size_t)units_per_layer * chunk * sizeof(int32_t),
                    "cudaMalloc(unit flags)")) != TRI_OK)
         return st;
+
     const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
     if ((st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
     if ((st = launch_validate(c, kv, t, mode, cap_u, c->d_seq_bad, stream)) != TRI_OK) return st;
@@ -728,8 +734,11 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
         ce = cudaLaunchKernelEx(&cfg, score_fn, tmap, m);
         if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx(score)");
         const bool last = lr0 + nl == kv->n_layers;
-        st = launch_fused(c, fused, &sub, t, budget, raw_c, zmax_c, mode, cap_u, c->d_pre, c->d_unit_fail,
-                          m.unit_base, (finalize && last) ? kv->lens_out : nullptr, c->d_seq_bad, stream);
+        PreScores ps;
+        ps.scores = c->d_pre;
+        ps.unit_fail = c->d_unit_fail;
+        st = launch_fused(c, fused, &sub, t, budget, raw_c, zmax_c, mode, cap_u, ps, m.unit_base,
+                          (finalize && last) ? kv->lens_out : nullptr, c->d_seq_bad, stream);
         if (st != TRI_OK) return st;
     }
     return TRI_OK;
@@ -757,7 +766,7 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
     const bool finalize = mode == tri::kModePrune && kv->lens_out != nullptr;
     if ((st = ensure_seq_bad(c, kv->batch)) != TRI_OK) return st;
     if ((st = launch_validate(c, kv, t, mode, cap_u, c->d_seq_bad, stream)) != TRI_OK) return st;
-    return launch_fused(c, fn, kv, t, budget, raw, zmax, mode, cap_u, nullptr, nullptr, 0,
+    return launch_fused(c, fn, kv, t, budget, raw, zmax, mode, cap_u, PreScores(), 0,
                         finalize ? kv->lens_out : nullptr, c->d_seq_bad, stream);
 }
 
@@ -971,19 +980,26 @@ tri_status run_attend(tri_ctx *c, const tri_kv *kv, const void *q, float *out, v
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
 
-    // launch shape: the deepest per-warp ring (3 stages at most) that keeps two CTAs per SM
-    int nslot = 3, per_sm = 0;
-    for (; nslot >= 1; --nslot) {
-        const size_t smem = tri::att_smem_bytes(c->D, c->G, nslot);
-        ce = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute(attend)");
-        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, tri::kAttThreads, smem) != cudaSuccess) {
+    // launch shape: the deepest per-warp ring (3 stages at most) that keeps three CTAs per SM,
+    // else the ring depth that gives the most CTAs per SM (registers may allow only two)
+    ce = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)tri::att_smem_bytes(c->D, c->G, 3));
+    if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaFuncSetAttribute(attend)");
+    int nslot = 0, per_sm = 0;
+    for (int ns = 3; ns >= 1; --ns) {
+        int p = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p, fn, tri::kAttThreads,
+                                                          tri::att_smem_bytes(c->D, c->G, ns)) != cudaSuccess) {
             cudaGetLastError();
-            per_sm = 0;
+            continue;
         }
-        if (per_sm >= 2 || nslot == 1) break;
+        if (p > per_sm) {
+            per_sm = p;
+            nslot = ns;
+        }
+        if (p >= 3) break;
     }
-    if (per_sm < 1) return TRI_EUNSUPPORTED;
+    if (per_sm < 1 || nslot < 1) return TRI_EUNSUPPORTED;
     // chunks per unit: split the units' rows only when there are too few units for four waves
     const long long target = 4LL * c->sm_count * per_sm;
     long long cpu = (target + n_units - 1) / n_units;

@@ -96,7 +96,7 @@ struct Args {
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
     int32_t *seq_bad;            // [batch] sequences the device refused this call
-    const float *pre;            // precomputed scores [n_units][cap_u][G] (max-over-offsets mode)
+    const float *pre;            // precomputed scores [n_units][cap_u][G] (tensor-core engine)
     const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing
     long long unit_base;         // added to the unit index in device status reports
     int wait_tries;              // tries (about 1 ms each) of every bounded wait

@@ -297,11 +297,19 @@ __global__ void __launch_bounds__(256) tri_mx_image_kernel(const MxArgs a) {
         const __nv_bfloat16 ih = __float2bfloat16_rn((float)im);
         const __nv_bfloat16 rl = __float2bfloat16_rn((float)(re - (double)__bfloat162float(rh)));
         const __nv_bfloat16 il = __float2bfloat16_rn((float)(im - (double)__bfloat162float(ih)));
-        const unsigned ore = mx_swz_offset(n, dre, ncol) / 2u, oim = mx_swz_offset(n, dim, ncol) / 2u;
-        hi[ore] = rh;
-        hi[oim] = ih;
-        lo[ore] = rl;
-        lo[oim] = il;
+        if (a.noffp == 1) {
+            // one operand of 2 ncol rows per chunk: hi rows, then lo rows (a single MMA reads both)
+            hi[mx_swz_offset(n, dre, 2 * ncol) / 2u] = rh;
+            hi[mx_swz_offset(n, dim, 2 * ncol) / 2u] = ih;
+            hi[mx_swz_offset(ncol + n, dre, 2 * ncol) / 2u] = rl;
+            hi[mx_swz_offset(ncol + n, dim, 2 * ncol) / 2u] = il;
+        } else {
+            const unsigned ore = mx_swz_offset(n, dre, ncol) / 2u, oim = mx_swz_offset(n, dim, ncol) / 2u;
+            hi[ore] = rh;
+            hi[oim] = ih;
+            lo[ore] = rl;
+            lo[oim] = il;
+        }
     }
     float *w = reinterpret_cast<float *>(img + 2u * half);
     for (int idx = threadIdx.x; idx < G * F; idx += blockDim.x) {
@@ -336,7 +344,11 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     constexpr int KCH = D / 64;         // 64-dim chunks (128-byte rows)
     constexpr int KSTEPS = D / 16;      // MMA k-steps per tile
     constexpr int NCOL = mx_ncol(G, NOFF);
-    constexpr int ACC = mx_acc_cols(NCOL);
+    // one column per head: hi and lo coefficients form one operand of 2 NCOL rows, so one MMA
+    // per k-step reads the key tile once; the epilogue adds the two halves of the accumulator
+    constexpr bool CAT = NOFF == 1;
+    constexpr int NMMA = CAT ? 2 * NCOL : NCOL;
+    constexpr int ACC = mx_acc_cols(NMMA);
     constexpr int NACC = mx_nacc(ACC);
     constexpr int NE = kMxEpiGroups;
     constexpr int REAL = G * NOFF;      // columns that hold a (head, offset) score
@@ -492,7 +504,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     } else if (warp == 1) {
         // ---------------- MMA issuer ----------------
         if (lane == 0) {
-            const uint32_t idesc = mx_idesc(NCOL);
+            const uint32_t idesc = mx_idesc(NMMA);
             MxWalk wk;
             wk.start(a, T0, per_layer);
             int seg = -1, prev_unit = -1;
@@ -526,10 +538,15 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 for (int ks = 0; ks < KSTEPS; ++ks) {
                     const unsigned koff = (unsigned)(ks & 3) * 32u;  // K = 16 bf16 = 32 bytes per step
                     const uint64_t ad = mx_desc(As + (ks >> 2) * kMxChunkBytes + koff);
-                    const uint64_t bh = mx_desc(Bs + (unsigned)(ks >> 2) * NCOL * 128u + koff);
-                    const uint64_t bl = mx_desc(Bs + half + (unsigned)(ks >> 2) * NCOL * 128u + koff);
-                    mx_mma(dt, ad, bh, idesc, ks > 0 ? 1 : 0);
-                    mx_mma(dt, ad, bl, idesc, 1);
+                    if constexpr (CAT) {
+                        const uint64_t bc = mx_desc(Bs + (unsigned)(ks >> 2) * NMMA * 128u + koff);
+                        mx_mma(dt, ad, bc, idesc, ks > 0 ? 1 : 0);
+                    } else {
+                        const uint64_t bh = mx_desc(Bs + (unsigned)(ks >> 2) * NCOL * 128u + koff);
+                        const uint64_t bl = mx_desc(Bs + half + (unsigned)(ks >> 2) * NCOL * 128u + koff);
+                        mx_mma(dt, ad, bh, idesc, ks > 0 ? 1 : 0);
+                        mx_mma(dt, ad, bl, idesc, 1);
+                    }
                 }
                 mx_commit(accfull + ab);
                 if (k + 1 == count || wk.last_of_unit()) mx_commit(bempty + (seg & 1));
@@ -633,8 +650,18 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
 #pragma unroll
                 for (int h = 0; h < G; ++h) best[h] = __int_as_float(0xff800000);
                 const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * ACC);
+                if constexpr (CAT) {
+                    // columns [0, G): the hi products, [NCOL, NCOL + G): the lo products
+                    uint32_t v0[16], v1[16];
+                    tmem_ld16_issue(tbase, v0);
+                    tmem_ld16_issue(tbase + (uint32_t)NCOL, v1);
+                    tmem_wait_ld(v0);
+                    tmem_after_wait(v1);
 #pragma unroll
-                for (int c0 = 0; c0 < REAL; c0 += 32) {
+                    for (int h = 0; h < G; ++h) best[h] = __uint_as_float(v0[h]) + __uint_as_float(v1[h]);
+                }
+#pragma unroll
+                for (int c0 = 0; c0 < (CAT ? 0 : REAL); c0 += 32) {
                     uint32_t v0[16], v1[16];
                     tmem_ld16_issue(tbase + (uint32_t)c0, v0);
                     if (c0 + 16 < REAL) tmem_ld16_issue(tbase + (uint32_t)(c0 + 16), v1);
@@ -667,10 +694,11 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                     mbar_arrive(empty + stage);
                 }
                 const int key = wk.tile * kMxTile + r;
-                if (key < wk.N) {
-                    float sv[G];
+                const bool valid = key < wk.N;
+                float sv[G];
 #pragma unroll
-                    for (int h = 0; h < G; ++h) sv[h] = best[h] + (nrm[h].x + nrm[h].y);
+                for (int h = 0; h < G; ++h) sv[h] = best[h] + (nrm[h].x + nrm[h].y);
+                if (valid) {
                     float *dst = a.pre + ((long long)unit * a.cap_u + key) * G;
                     if constexpr (G >= 4) {
 #pragma unroll

@@ -68,6 +68,46 @@ def test_noalloc_matches_prune_on_two_calls():
     ctx.close()
 
 
+def test_noalloc_refusal_does_not_carry_over():
+    """The sequence-level verdicts of the allocation-free prune live in the fixed flag array: a
+    sequence refused on one call (a cached position not below t) is left untouched, and the
+    next call, on a clean copy, prunes it like tri_prune does."""
+    spec = ts.CacheSpec(name="noalloc_refuse", head_dim=128, group=4, n_kv_heads=2, n_layers=2, batch=3,
+                        rope_base=1e6, budget=100, offsets=ts.pow2_offsets(16), positions="from_zero",
+                        lens=(300, 250, 410), key_sigma=(0.1, 0.6), cap=448)
+    base = ts.make_cache(spec, 33).to("cuda")
+    U = base.n_units
+    rows_in = [base.unit_rows(u) for u in range(U)]
+    ctx = gu.context_for(base)
+    ref = base.clone()
+    ctx.prune(ref.K, ref.V, ref.pos, ref.lens, ref.t, spec.budget)
+    assert ctx.get_error()[0] == tri.TRI_OK
+
+    bad = base.clone()
+    bad.pos[1, 1, 0, spec.lens[1] - 1] = int(bad.t_host[1])  # layer 1, sequence 1, KV head 0
+    bad_rows = [bad.unit_rows(u) for u in range(U)]
+    ctx.prune_noalloc(bad.K, bad.V, bad.pos, bad.lens, bad.t, spec.budget)
+    st, code, unit = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == tri.TRI_DEV_T_NOT_AFTER_POS
+    assert bad.unit_index(unit)[1] == 1
+    assert bad.lens_host.tolist() == [100, 250, 100]
+    for u in range(U):
+        if bad.unit_index(u)[1] == 1:
+            out = gu.unit_output_rows(bad, u, spec.lens[1])
+            assert all(np.array_equal(x, y) for x, y in zip(out, bad_rows[u])), u
+
+    clean = base.clone()
+    ctx.prune_noalloc(clean.K, clean.V, clean.pos, clean.lens, clean.t, spec.budget)
+    assert ctx.get_error()[0] == tri.TRI_OK
+    assert np.array_equal(clean.lens_host, ref.lens_host)
+    for u in range(U):
+        out = clean.unit_rows(u)
+        kept = _kept_slots(rows_in[u], out)
+        assert np.array_equal(kept, _kept_slots(rows_in[u], ref.unit_rows(u))), u
+        gu.check_compacted(rows_in[u], out, kept, f"unit {u}")
+    ctx.close()
+
+
 def test_noalloc_limits_are_rejected_without_launch():
     # a unit capacity of 2^21 slots: no launch shape keeps its keep mask on chip, so both entry
     # points refuse it (for every capacity tri_prune accepts, one score slot stays far below the
