@@ -728,7 +728,7 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
         cudaLaunchConfig_t cfg;
         std::memset(&cfg, 0, sizeof cfg);
         cfg.gridDim = dim3((unsigned)c->sm_count);
-        cfg.blockDim = dim3((unsigned)tri::kMxThreads);
+        cfg.blockDim = dim3((unsigned)tri::mx_threads(G, noffp));
         cfg.dynamicSmemBytes = smem;
         cfg.stream = cs;
         ce = cudaLaunchKernelEx(&cfg, score_fn, tmap, m);

@@ -23,7 +23,7 @@
 //             about 16 significant bits of C while the key stays exact.
 //   MMA       per 128-key tile: d/16 k-steps, each an M=128, N=NCOL, K=16 MMA for hi and one
 //             for lo, both accumulating into the same fp32 TMEM accumulator.
-//   epilogue  two warpgroups of 4 warps take the tiles in turn, one TMEM lane (key) per
+//   epilogue  warpgroups of 4 warps take the tiles in turn, one TMEM lane (key) per
 //             thread: the max over each head's columns (a head owns NOFF consecutive columns,
 //             NOFF a compile-time count, the last offset repeated when the set is smaller,
 //             so the max unrolls into three-input max instructions), plus the norm score from
@@ -32,10 +32,11 @@
 //             compaction read instead of scoring the keys themselves.
 //
 // One CTA per SM, warp-specialised: warp 0 issues the TMA loads, warp 1 owns the TMEM
-// allocation and issues the MMAs, warps 2-9 run the epilogue. Key tiles stream through a
-// ring of NST stages; up to four accumulators live in TMEM (tile k in buffer k mod NACC, its
-// epilogue in warpgroup k mod 2); the coefficient image is double-buffered in shared memory
-// and reloaded only when the CTA's tile range enters a new unit.
+// allocation and issues the MMAs, the other warps (three warpgroups, or two where the TMEM
+// holds only two accumulators) run the epilogue. Key tiles stream through a ring of NST
+// stages; the accumulators live in TMEM (tile k in buffer k mod NACC, its epilogue in
+// warpgroup k mod NE); the coefficient image is double-buffered in shared memory and reloaded
+// only when the CTA's tile range enters a new unit.
 //
 // The same kernel scores the mean over the offsets on the tensor cores (NOFF = 1): the
 // coefficient of a head is then qbar A_f e^{i omega_f t}, the offset average folded in. Every wait is bounded; a wait that runs out records a device status, marks every unit
@@ -52,8 +53,10 @@
 
 namespace tri {
 
-constexpr int kMxEpiGroups = 2;                         // epilogue warpgroups (tiles in turn)
-constexpr int kMxThreads = 64 + 128 * kMxEpiGroups;     // warp 0: TMA, warp 1: MMA + TMEM, then the epilogue
+// Epilogue warpgroups (taking the tiles in turn): three where the TMEM holds three accumulators,
+// else two. Threads per CTA: warp 0 issues the TMA loads, warp 1 the MMAs, then the epilogue.
+__host__ __device__ constexpr int mx_epi_groups(int acc_cols) { return 512 / acc_cols >= 3 ? 3 : 2; }
+__host__ __device__ constexpr int mx_threads_of(int acc_cols) { return 64 + 128 * mx_epi_groups(acc_cols); }
 constexpr int kMxTile = 128;       // keys per tile (the MMA's M)
 constexpr int kMxMaxStages = 6;
 constexpr unsigned kMxChunkBytes = kMxTile * 128u;  // one 64-dim chunk of a tile: 128 rows x 128 B
@@ -68,9 +71,15 @@ __host__ __device__ constexpr int mx_ncol(int G, int noff) { return (G * noff + 
 __host__ __device__ constexpr int mx_acc_cols(int ncol) {
     return ncol <= 32 ? 32 : ncol <= 64 ? 64 : ncol <= 128 ? 128 : 256;
 }
-// Accumulator buffers: as many as 512 TMEM columns hold, at most 4 (a multiple of the
-// epilogue warpgroups, so that one warpgroup owns every tile of a buffer).
-__host__ __device__ constexpr int mx_nacc(int acc_cols) { return 512 / acc_cols < 4 ? 512 / acc_cols : 4; }
+// Accumulator buffers: one per epilogue warpgroup (so that one warpgroup owns every tile of a
+// buffer), two per warpgroup where the 512 TMEM columns allow it.
+__host__ __device__ constexpr int mx_nacc(int acc_cols) {
+    return 512 / acc_cols >= 2 * mx_epi_groups(acc_cols) ? 2 * mx_epi_groups(acc_cols) : mx_epi_groups(acc_cols);
+}
+// Threads of the scoring kernel for head_dim-independent geometry (group, columns per head).
+__host__ __device__ constexpr int mx_threads(int G, int noff) {
+    return mx_threads_of(mx_acc_cols(noff == 1 ? 2 * mx_ncol(G, noff) : mx_ncol(G, noff)));
+}
 // Bytes of one half (hi or lo) of a coefficient image: d/64 chunks of NCOL rows x 128 B.
 __host__ __device__ constexpr unsigned mx_half_bytes(int D, int ncol) { return (unsigned)(D / 64) * ncol * 128u; }
 // Whole image: hi, lo, then the norm weights [G][F] fp32; a multiple of 1024 bytes.
@@ -338,7 +347,7 @@ __host__ __device__ inline MxLayout mx_layout(int D, int G, int ncol, int nst) {
 // The scoring kernel. NOFF: columns per head (mx_noff_pad of the offset count).
 // ---------------------------------------------------------------------------------
 template <int D, int G, int LAYOUT, int NOFF>
-__global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __grid_constant__ CUtensorMap tmap,
+__global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(const __grid_constant__ CUtensorMap tmap,
                                                                      const MxArgs a) {
     constexpr int F = D / 2;
     constexpr int KCH = D / 64;         // 64-dim chunks (128-byte rows)
@@ -350,7 +359,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
     constexpr int NMMA = CAT ? 2 * NCOL : NCOL;
     constexpr int ACC = mx_acc_cols(NMMA);
     constexpr int NACC = mx_nacc(ACC);
-    constexpr int NE = kMxEpiGroups;
+    constexpr int NE = mx_epi_groups(ACC);
     constexpr int REAL = G * NOFF;      // columns that hold a (head, offset) score
     static_assert(NACC % NE == 0 && NACC * ACC <= 512, "accumulator buffers");
     constexpr unsigned kStageBytes = KCH * kMxChunkBytes;
@@ -396,7 +405,9 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
         *abort_flag = 0;
         mbar_init_fence();
     }
-    constexpr unsigned kTmemCols = (unsigned)(NACC * ACC) < 32u ? 32u : (unsigned)(NACC * ACC);
+    // a TMEM allocation is a power of two of at least 32 columns
+    constexpr unsigned kTmemCols = NACC * ACC <= 32 ? 32u : NACC * ACC <= 64 ? 64u : NACC * ACC <= 128 ? 128u
+                                                          : NACC * ACC <= 256 ? 256u : 512u;
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_holder)),
                      "r"(kTmemCols)
@@ -602,7 +613,7 @@ __global__ void __launch_bounds__(kMxThreads, 1) tri_mx_score_kernel(const __gri
                 float2 nrm[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) nrm[h] = make_float2(0.f, 0.f);
-#pragma unroll
+#pragma unroll 2
                 for (int f0 = 0; f0 < F; f0 += 8) {
                     // band moduli of bands f0 .. f0 + 7, as four pairs (f, f + 1)
                     float2 nb[4];
