@@ -237,8 +237,9 @@ TRI_API tri_status tri_prune(tri_ctx *ctx, const tri_kv *kv, const int32_t *t, i
  * its scratch.)
  *   Same arguments, semantics and results as tri_prune. The scores of the units in flight live
  *   in a fixed 64 MiB device array that the library holds on every GPU that loads it, until the
- *   process exits; sequences the device refuses are flagged in a fixed array of 16384 entries.
- *   It calls no cudaMalloc or cudaFree; it zeroes the flags with cudaMemsetAsync on `stream`.
+ *   process exits; the validation kernel writes every sequence's verdict (0 when accepted) into
+ *   a fixed array of 16384 entries on every call, so nothing needs clearing beforehand. It
+ *   calls no cudaMalloc, cudaFree or allocating library routine.
  * Limits: batch <= 16384; the unit-capacity limit of tri_prune applies unchanged (within it
  *   one unit's score slot, capacity * (group + 1) floats, stays below 19 MB). When the 64 MiB
  *   holds fewer slots than tri_prune would run clusters, fewer clusters run: same results, a

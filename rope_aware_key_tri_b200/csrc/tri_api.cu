@@ -774,11 +774,11 @@ tri_status run(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budget, f
 // Allocation-free prune. Some callers cannot allocate device memory at call time: a serving
 // loop whose device memory is owned by another allocator, or one that cannot afford the
 // device-wide synchronisation that cudaFree implies when tri_prune has to grow its scratch.
-// For them the per-cluster score slots (and the per-sequence refusal flags) live in
+// For them the per-cluster score slots (and the per-sequence validation verdicts) live in
 // file-scope device arrays of fixed size, loaded with the library and held until exit.
 // ---------------------------------------------------------------------------------------
 constexpr size_t kNoAllocScratchBytes = size_t(64) << 20;  // score slots: 64 MiB
-constexpr int kNoAllocMaxBatch = 16384;                       // refusal flags
+constexpr int kNoAllocMaxBatch = 16384;                       // validation verdicts
 constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchBytes / sizeof(float)];

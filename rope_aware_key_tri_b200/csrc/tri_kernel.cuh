@@ -95,7 +95,7 @@ struct Args {
     long long slot_floats;       // floats per slot
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
-    int32_t *seq_bad;            // [batch] sequences the device refused this call
+    int32_t *seq_bad;            // [batch] the validation kernel's verdicts (0: accepted)
     const float *pre;            // precomputed scores [n_units][cap_u][G] (tensor-core engine)
     const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing
     long long unit_base;         // added to the unit index in device status reports

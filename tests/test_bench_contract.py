@@ -30,3 +30,17 @@ def test_reference_arm_json_line(combine):
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == j["value"]
     e2e = j["e2e"]
     assert e2e["value"] == j["value"] and e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+def test_traffic_figure_follows_the_code_not_its_comments():
+    """roofline.traffic comes from a committed ncu summary only while the prune kernel's code is
+    the one the counters were taken on: the hash ignores comments and layout, not code."""
+    sys.path.insert(0, ROOT)
+    import bench
+    a = "int f(int x) { // doubles x\n  return 2 * x; /* fast */ }\nconst char *s = \"a//b\";"
+    b = "int f(int x)\n{\n  return 2 * x;\n}\nconst char *s = \"a//b\";  // other words"
+    c = "int f(int x) { return 3 * x; } const char *s = \"a//b\";"
+    assert bench._code_only(a) == bench._code_only(b)
+    assert bench._code_only(a) != bench._code_only(c)
+    assert "a//b" in bench._code_only(a)
+    assert len(bench.kernel_source_hash()) == 16
