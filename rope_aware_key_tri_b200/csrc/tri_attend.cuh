@@ -216,19 +216,29 @@ __global__ void __launch_bounds__(kAttThreads) tri_attend_kernel(const AttArgs a
 #pragma unroll
                 for (int h = 0; h < G; ++h) sv[pp][h] = r < valid ? dsum[h] : NEG_INF;
             }
+            // the running maxima only move when a logit of this sub-block exceeds them, which
+            // after the first few sub-blocks is rare: the warp rescales only when some lane's did
+            float mnew[G];
+            bool grew = false;
 #pragma unroll
             for (int h = 0; h < G; ++h) {
                 float mb = sv[0][h];
 #pragma unroll
                 for (int pp = 1; pp < SB; ++pp) mb = fmaxf(mb, sv[pp][h]);
-                const float mn = fmaxf(m[h], mb);
-                if (mn != NEG_INF) {
-                    const float corr = ex2_approx(m[h] - mn);  // 0 while m is still -inf
-                    l[h] *= corr;
-                    const float2 c2 = make_float2(corr, corr);
+                mnew[h] = fmaxf(m[h], mb);
+                grew |= mnew[h] > m[h];
+            }
+            if (__any_sync(FULL, grew)) {
 #pragma unroll
-                    for (int i = 0; i < DPL / 2; ++i) acc[h][i] = __fmul2_rn(acc[h][i], c2);
-                    m[h] = mn;
+                for (int h = 0; h < G; ++h) {
+                    if (mnew[h] != NEG_INF) {
+                        const float corr = ex2_approx(m[h] - mnew[h]);  // 1 if unchanged, 0 from -inf
+                        l[h] *= corr;
+                        const float2 c2 = make_float2(corr, corr);
+#pragma unroll
+                        for (int i = 0; i < DPL / 2; ++i) acc[h][i] = __fmul2_rn(acc[h][i], c2);
+                        m[h] = mnew[h];
+                    }
                 }
             }
 #pragma unroll

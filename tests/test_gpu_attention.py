@@ -149,3 +149,39 @@ def test_attention_refused_sequence_is_not_written():
     o[:, 1] = 0.0
     check_attention(cache, q, o, lens=lens, label="others")
     ctx.close()
+
+
+@pytest.mark.parametrize("page_size", [32, 48])
+def test_attention_paged_odd_pages(page_size):
+    """Pages of 32 and 48 slots (GQA 8): a 16-row stage never crosses a page."""
+    spec = ts.replace(ts.WORKLOADS["qwen3_32b_paged_ragged"], n_layers=1, batch=3, lens=(400, 257, 48),
+                      page_size=page_size, budget=100, cap=480)
+    cache = ts.make_cache(spec, 50).to("cuda")
+    q = _queries(spec, 51)
+    ctx = gu.context_for(cache)
+    out = ctx.decode_attention(cache.K, cache.V, cache.lens, q, block_table=cache.block_table)
+    assert ctx.get_error()[0] == tri.TRI_OK
+    check_attention(cache, q, out, label=f"paged{page_size}")
+    ctx.close()
+
+
+def test_attention_layer_range():
+    """A call on a sub-range of the layers (layer_begin) attends over exactly those layers (its
+    units may be split into chunks differently from a full call, so each result is checked
+    against the oracle, not against the other bit for bit)."""
+    spec = ts.CacheSpec(name="att_layers", head_dim=128, group=4, n_kv_heads=2, n_layers=3, batch=2,
+                        rope_base=1e6, budget=64, offsets=(1,), positions="from_zero",
+                        lens=(300, 77), key_sigma=(0.1, 0.6), cap=320)
+    cache = ts.make_cache(spec, 52).to("cuda")
+    q = _queries(spec, 53)
+    ctx = gu.context_for(cache)
+    full = ctx.decode_attention(cache.K, cache.V, cache.lens, q)
+    part = ctx.decode_attention(cache.K[1:3].contiguous(), cache.V[1:3].contiguous(), cache.lens,
+                                q[1:3].contiguous(), layer_begin=1)
+    assert ctx.get_error()[0] == tri.TRI_OK
+    check_attention(cache, q, full, label="all layers")
+    sub = ts.Cache(ts.replace(spec, n_layers=2), cache.K[1:3], cache.V[1:3], cache.pos[1:3], cache.lens,
+                   cache.t, None, 0, cache.cap, (cache.q_mean[1:3], cache.q_norm_mean[1:3], cache.R[1:3],
+                                                 cache.offsets))
+    check_attention(sub, q[1:3], part, label="layers 1-2")
+    ctx.close()
