@@ -173,6 +173,22 @@ __device__ __forceinline__ void tmem_ld16_issue(uint32_t taddr, uint32_t (&r)[16
         : "memory");
 }
 
+// 8 accumulator columns, without waiting (valid after tmem_wait_ld8 on the same registers).
+__device__ __forceinline__ void tmem_ld8_issue(uint32_t taddr, uint32_t (&r)[8]) {
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+                 : "r"(taddr)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld8(uint32_t (&a)[8], uint32_t (&b)[8]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(a[0]), "+r"(a[1]), "+r"(a[2]), "+r"(a[3]), "+r"(a[4]), "+r"(a[5]), "+r"(a[6]), "+r"(a[7]),
+                   "+r"(b[0]), "+r"(b[1]), "+r"(b[2]), "+r"(b[3]), "+r"(b[4]), "+r"(b[5]), "+r"(b[6]), "+r"(b[7])
+                 :
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[16]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;"
                  : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
@@ -602,6 +618,21 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                     if (lane == 0) fail(unit);
                     break;
                 }
+                // one column per head: the accumulator (usually complete by now: the MMA warp runs
+                // ahead) is read while the norm term is computed, so the TMEM latency overlaps it
+                uint32_t acc_hi[8], acc_lo[8];
+                if constexpr (CAT) {
+                    const bool ok_acc0 = __all_sync(
+                        0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
+                    if (!ok_acc0) {
+                        if (lane == 0) fail(unit);
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t tb = tmem_base + lane_base + (uint32_t)(ab * ACC);
+                    tmem_ld8_issue(tb, acc_hi);
+                    tmem_ld8_issue(tb + (uint32_t)NCOL, acc_lo);
+                }
                 const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
                 const float *wsm =
                     reinterpret_cast<const float *>(smem + Ly.image + (seg & 1) * img_bytes + 2u * half);
@@ -649,13 +680,15 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                     }
                 }
 
-                const bool ok_acc =
-                    __all_sync(0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
-                if (!ok_acc) {
-                    if (lane == 0) fail(unit);
-                    break;
+                if constexpr (!CAT) {
+                    const bool ok_acc = __all_sync(
+                        0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
+                    if (!ok_acc) {
+                        if (lane == 0) fail(unit);
+                        break;
+                    }
+                    tc_fence_after();
                 }
-                tc_fence_after();
                 // max over each head's NOFF columns: 32 columns per wait
                 float best[G];
 #pragma unroll
@@ -663,13 +696,9 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                 const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * ACC);
                 if constexpr (CAT) {
                     // columns [0, G): the hi products, [NCOL, NCOL + G): the lo products
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16_issue(tbase, v0);
-                    tmem_ld16_issue(tbase + (uint32_t)NCOL, v1);
-                    tmem_wait_ld(v0);
-                    tmem_after_wait(v1);
+                    tmem_wait_ld8(acc_hi, acc_lo);
 #pragma unroll
-                    for (int h = 0; h < G; ++h) best[h] = __uint_as_float(v0[h]) + __uint_as_float(v1[h]);
+                    for (int h = 0; h < G; ++h) best[h] = __uint_as_float(acc_hi[h]) + __uint_as_float(acc_lo[h]);
                 }
 #pragma unroll
                 for (int c0 = 0; c0 < (CAT ? 0 : REAL); c0 += 32) {
