@@ -376,6 +376,8 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
     constexpr int ACC = mx_acc_cols(NMMA);
     constexpr int NACC = mx_nacc(ACC);
     constexpr int NE = mx_epi_groups(ACC);
+    constexpr bool EARLY = NACC >= 2 * NE;                // the MMA warp can run a tile ahead
+    constexpr int NCH = CAT ? 0 : (G * NOFF + 31) / 32;  // 32-column chunks of the max
     constexpr int REAL = G * NOFF;      // columns that hold a (head, offset) score
     static_assert(NACC % NE == 0 && NACC * ACC <= 512, "accumulator buffers");
     constexpr unsigned kStageBytes = KCH * kMxChunkBytes;
@@ -618,10 +620,27 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                     if (lane == 0) fail(unit);
                     break;
                 }
-                // one column per head: the accumulator (usually complete by now: the MMA warp runs
-                // ahead) is read while the norm term is computed, so the TMEM latency overlaps it
+                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * ACC);
+                // accumulator columns are read in chunks of 32, each chunk's load issued before the
+                // previous chunk is reduced; one column per head takes 8 hi and 8 lo columns
                 uint32_t acc_hi[8], acc_lo[8];
-                if constexpr (CAT) {
+                uint32_t pa[16], pb[16], qa[16], qb[16];
+                auto issue_chunk = [&](int c, uint32_t(&x)[16], uint32_t(&y)[16]) {
+                    tmem_ld16_issue(tbase + (uint32_t)(32 * c), x);
+                    if (32 * c + 16 < REAL) tmem_ld16_issue(tbase + (uint32_t)(32 * c + 16), y);
+                };
+                auto issue_first = [&]() {
+                    if constexpr (CAT) {
+                        tmem_ld8_issue(tbase, acc_hi);
+                        tmem_ld8_issue(tbase + (uint32_t)NCOL, acc_lo);
+                    } else {
+                        issue_chunk(0, pa, pb);
+                    }
+                };
+                // where the MMA warp runs a tile ahead of this warpgroup (two accumulators each), the
+                // accumulator is usually complete by now, and its first chunk is read while the norm
+                // term is computed; otherwise the norm term overlaps the tile's MMAs instead
+                if constexpr (EARLY) {
                     const bool ok_acc0 = __all_sync(
                         0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
                     if (!ok_acc0) {
@@ -629,9 +648,7 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t tb = tmem_base + lane_base + (uint32_t)(ab * ACC);
-                    tmem_ld8_issue(tb, acc_hi);
-                    tmem_ld8_issue(tb + (uint32_t)NCOL, acc_lo);
+                    issue_first();
                 }
                 const unsigned char *As = smem + Ly.stage + (unsigned)stage * kStageBytes;
                 const float *wsm =
@@ -680,7 +697,7 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                     }
                 }
 
-                if constexpr (!CAT) {
+                if constexpr (!EARLY) {
                     const bool ok_acc = __all_sync(
                         0xffffffffu, mbar_wait_bounded(accfull + ab, (unsigned)((k / NACC) & 1), a.wait_tries));
                     if (!ok_acc) {
@@ -688,30 +705,24 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                         break;
                     }
                     tc_fence_after();
+                    issue_first();
                 }
-                // max over each head's NOFF columns: 32 columns per wait
+                // max over each head's NOFF columns
                 float best[G];
 #pragma unroll
                 for (int h = 0; h < G; ++h) best[h] = __int_as_float(0xff800000);
-                const uint32_t tbase = tmem_base + lane_base + (uint32_t)(ab * ACC);
                 if constexpr (CAT) {
                     // columns [0, G): the hi products, [NCOL, NCOL + G): the lo products
                     tmem_wait_ld8(acc_hi, acc_lo);
 #pragma unroll
                     for (int h = 0; h < G; ++h) best[h] = __uint_as_float(acc_hi[h]) + __uint_as_float(acc_lo[h]);
                 }
-#pragma unroll
-                for (int c0 = 0; c0 < (CAT ? 0 : REAL); c0 += 32) {
-                    uint32_t v0[16], v1[16];
-                    tmem_ld16_issue(tbase + (uint32_t)c0, v0);
-                    if (c0 + 16 < REAL) tmem_ld16_issue(tbase + (uint32_t)(c0 + 16), v1);
-                    tmem_wait_ld(v0);
-                    if (c0 + 16 < REAL) tmem_after_wait(v1);
+                auto reduce_chunk = [&](int c, const uint32_t(&v0)[16], const uint32_t(&v1)[16]) {
                     // columns pair up within a head (offsets 2j, 2j + 1) for one three-input max;
                     // every index below is a compile-time constant once the loops unroll
 #pragma unroll
                     for (int i = 0; i < 32; ++i) {
-                        const int col = c0 + i;
+                        const int col = 32 * c + i;
                         if (col < REAL) {
                             const int h = col / NOFF, j = col - h * NOFF;
                             const float x = __uint_as_float(i < 16 ? v0[i] : v1[i - 16]);
@@ -724,6 +735,21 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
                                 best[h] = fmaxf(best[h], x);
                             }
                         }
+                    }
+                };
+#pragma unroll
+                for (int c = 0; c < NCH; ++c) {
+                    const bool two = 32 * c + 16 < REAL;
+                    if (c % 2 == 0) {
+                        tmem_wait_ld(pa);
+                        if (two) tmem_after_wait(pb);
+                        if (c + 1 < NCH) issue_chunk(c + 1, qa, qb);
+                        reduce_chunk(c, pa, pb);
+                    } else {
+                        tmem_wait_ld(qa);
+                        if (two) tmem_after_wait(qb);
+                        if (c + 1 < NCH) issue_chunk(c + 1, pa, pb);
+                        reduce_chunk(c, qa, qb);
                     }
                 }
                 tc_fence_before();
