@@ -530,6 +530,7 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     a.pre = pre.scores;
     a.unit_fail = pre.unit_fail;
     a.unit_base = unit_base;
+    a.stagger = 1;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
@@ -900,6 +901,7 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     a.ring_extra = plan.extra;
     a.scratch = sym.scratch;
     a.slot_floats = slot_floats;
+    a.stagger = 1;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);

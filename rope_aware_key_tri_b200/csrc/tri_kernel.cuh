@@ -101,6 +101,7 @@ struct Args {
     long long unit_base;         // added to the unit index in device status reports
     int wait_tries;              // tries (about 1 ms each) of every bounded wait
     long long inject_unit;       // test hook: the unit whose first key copy is withheld (-1: none)
+    int stagger;                 // 1: clusters holding one unit fewer start half a unit period late
     unsigned *fail_count;        // units left uncompacted by a unit-level failure ...
     int32_t *fail_units;         // ... and the first fail_cap of them
     int fail_cap;
@@ -243,6 +244,29 @@ __device__ __forceinline__ void tma_load_1d(void *dst_smem, const void *src_gmem
 
 __device__ __forceinline__ void st_hint(float *p, float v, uint64_t policy) {
     asm volatile("st.global.L2::cache_hint.f32 [%0], %1, %2;" ::"l"(p), "f"(v), "l"(policy) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// The staggered start's wait (see the fused kernel); kept out of line, away from the kernel's
+// register allocation. Bounded by its own clock and by an iteration count.
+__device__ __noinline__ void stagger_wait(int n_units, int n_clusters, int cid, const int32_t *lens, int n_kv,
+                                          int batch, int cap_u, int budget, int D) {
+    const int q = n_units / n_clusters, r = n_units % n_clusters;
+    if (q < 2 || r == 0 || cid < r) return;
+    const int N0 = min(max(__ldg(lens + (cid / n_kv) % batch), 0), cap_u);
+    const float bytes = (float)N0 * (float)(2 * D) + (float)min(N0, budget) * (float)(8 * D + 8);
+    const unsigned long long wait_ns = (unsigned long long)(bytes * (float)n_clusters * (0.5f / 4600.f));
+    const unsigned long long t0 = global_ns();
+    for (int it = 0; it < (1 << 22) && global_ns() - t0 < wait_ns; ++it) __nanosleep(256);
+}
+
+__device__ __forceinline__ void prefetch_l1(const void *p) {
+    asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
 
 __device__ __forceinline__ void cp_async16(void *dst_smem, const void *src) {
@@ -577,6 +601,14 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     // set once a bounded wait of this cluster ran out: the ring's barrier phases can no longer
     // be trusted, so the cluster refuses its remaining units instead of streaming them
     bool dead = false;
+    // Staggered start. With n_units = q n_clusters + r (0 < r), clusters r.. hold one unit fewer
+    // and would idle at the end; they start about half a unit period late instead. Every
+    // cluster then meets the memory-bound phases (key stream, compaction) at a different time
+    // from the latency-bound ones (z-score, select, mask) of a fifth of the grid, where all
+    // clusters would otherwise reach each kind of phase together. The period is estimated from
+    // this cluster's first unit: its algorithmic bytes over the grid's share of 4.6 TB/s.
+    if (a.stagger && a.mode == kModePrune && !PRE)
+        stagger_wait(a.n_units, n_clusters, cid, a.lens, a.n_kv, a.batch, a.cap_u, a.budget, D);
     for (int unit = cid; unit < a.n_units; unit += n_clusters) {
         const int g = unit % a.n_kv;
         const int s = (unit / a.n_kv) % a.batch;
@@ -939,6 +971,12 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                     const int i = base + k * kThreads;
                     if (i < n_local) load_scores<G>(sc_read + (long long)i * G, sv[k]);
                 }
+                // the next batch is requested into L1 meanwhile (no registers held for it)
+#pragma unroll
+                for (int k = 0; k < ZB; ++k) {
+                    const int i = base + (ZB + k) * kThreads;
+                    if (i < n_local) prefetch_l1(sc_read + (long long)i * G);
+                }
 #pragma unroll
                 for (int k = 0; k < ZB; ++k) {
                     const int i = base + k * kThreads;
@@ -978,12 +1016,27 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                     for (int b = lane; b < kBins; b += 32) wh[b] = 0u;
                     __syncwarp();
                 }
-                // after the first digit few keys still match the prefix, and those spread over
-                // the bins: plain shared-memory atomics, no warp-level aggregation
+                // the matching keys spread over the bins: plain shared-memory atomics, no
+                // warp-level aggregation
+                auto count = [&](unsigned u, int i) {
+                    if (i < lim && (u & pmask) == prefix) atomicAdd(wh + ((u >> shift) & 255u), 1u);
+                };
+                if (keys_on_chip) {
+                    // four keys per 128-bit load, two loads in flight per thread
+                    const uint4 *u4 = reinterpret_cast<const uint4 *>(ring);
+                    const int n4 = (lim + 3) / 4;
+                    for (int j0 = tid; j0 < n4; j0 += 2 * kThreads) {
+                        const int j1 = j0 + kThreads;
+                        const uint4 x0 = u4[j0];
+                        const uint4 x1 = j1 < n4 ? u4[j1] : make_uint4(0u, 0u, 0u, 0u);
+                        count(x0.x, 4 * j0); count(x0.y, 4 * j0 + 1); count(x0.z, 4 * j0 + 2); count(x0.w, 4 * j0 + 3);
+                        if (j1 < n4) {
+                            count(x1.x, 4 * j1); count(x1.y, 4 * j1 + 1); count(x1.z, 4 * j1 + 2); count(x1.w, 4 * j1 + 3);
+                        }
+                    }
+                } else {
 #pragma unroll 4
-                for (int i = tid; i < lim; i += kThreads) {
-                    const unsigned u = uk[i];
-                    if ((u & pmask) == prefix) atomicAdd(wh + ((u >> shift) & 255u), 1u);
+                    for (int i = tid; i < lim; i += kThreads) count(uk[i], i);
                 }
                 __syncthreads();
                 unsigned *bh = bhist + (pass & 1) * kBins;
@@ -993,47 +1046,57 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                     bh[b] = c;
                 }
                 cluster.sync();
-                // global histogram, bins reversed so that index 0 is the top bin; every CTA
-                // folds the cluster's histograms in the same order and finds the same bin
-                for (int b = tid; b < kBins; b += kThreads) {
-                    unsigned part[kMaxCluster];
+                // global histogram in top-down order (index 0 = bin 255): thread t folds the
+                // cluster's counts of indices [t BPT, t BPT + BPT) in rank order, then a block
+                // scan finds the index whose running count first reaches `need` (every CTA
+                // folds in the same order and finds the same bin)
+                constexpr int BPT = (kBins + kThreads - 1) / kThreads;
+                int xs[BPT];
+                int tsum = 0;
 #pragma unroll
-                    for (int r = 0; r < kMaxCluster; ++r)
-                        part[r] = r < cs ? cluster.map_shared_rank(bh, r)[b] : 0u;
+                for (int j = 0; j < BPT; ++j) {
+                    const int idx = tid * BPT + j;
                     unsigned c = 0u;
+                    if (idx < kBins) {
+                        unsigned part[kMaxCluster];
 #pragma unroll
-                    for (int r = 0; r < kMaxCluster; ++r) c += part[r];
-                    gh[kBins - 1 - b] = (int)c;
+                        for (int r = 0; r < kMaxCluster; ++r)
+                            part[r] = r < cs ? cluster.map_shared_rank(bh, r)[kBins - 1 - idx] : 0u;
+#pragma unroll
+                        for (int r = 0; r < kMaxCluster; ++r) c += part[r];
+                    }
+                    xs[j] = (int)c;
+                    tsum += (int)c;
                 }
-                __syncthreads();
-                if (warp == 0) {
-                    int run = 0;
-                    for (int base = 0; base < kBins; base += 32) {
-                        const int x = gh[base + lane];
-                        int incl = x;
+                int incl = tsum;
 #pragma unroll
-                        for (int o = 1; o < 32; o <<= 1) {
-                            const int y = __shfl_up_sync(FULL, incl, o);
-                            if (lane >= o) incl += y;
-                        }
-                        incl += run;
-                        const int above = incl - x;
-                        if (above < need && incl >= need) {
-                            sel_s[0] = kBins - 1 - (base + lane);
-                            sel_s[1] = above;
-                            sel_s[2] = x;
-                        }
-                        run = __shfl_sync(FULL, incl, 31);
+                for (int o = 1; o < 32; o <<= 1) {
+                    const int y = __shfl_up_sync(FULL, incl, o);
+                    if (lane >= o) incl += y;
+                }
+                if (lane == 31) gh[warp] = incl;
+                __syncthreads();
+                int run = incl - tsum;
+                for (int w = 0; w < warp; ++w) run += gh[w];
+#pragma unroll
+                for (int j = 0; j < BPT; ++j) {
+                    const int above = run;
+                    run += xs[j];
+                    if (above < need && run >= need) {
+                        sel_s[0] = kBins - 1 - (tid * BPT + j);
+                        sel_s[1] = above;
+                        sel_s[2] = xs[j];
                     }
                 }
                 __syncthreads();
+                // gh and sel_s are next written after the next pass's cluster barrier, which
+                // every thread reaches only after reading them here: no trailing barrier
                 const int bstar = sel_s[0];
                 need -= sel_s[1];
                 const int cnt = sel_s[2];
                 prefix |= (unsigned)bstar << shift;
                 pmask |= 255u << shift;
                 resolved = (cnt == need);
-                __syncthreads();
             }
             const bool tie = !resolved;
 
@@ -1060,20 +1123,55 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                 __syncthreads();
                 tie_off = iscratch[kWarps + 1];
             }
-            for (int wi = warp; wi < nwl; wi += kWarps) {
-                const int i = wi * 32 + lane;
-                const bool in = i < n_local;
-                const unsigned u = in ? uk[i] : 0u;
-                const bool gt = in && (u & pmask) > prefix;
-                const bool eq = in && (u & pmask) == prefix;
-                bool keep = gt || (eq && !tie);
-                if (tie) {
-                    const unsigned eb = __ballot_sync(FULL, eq);
-                    const int rank = tie_off + tw[wi] + __popc(eb & ((1u << lane) - 1u));
-                    keep = gt || (eq && rank < need);
+            // Without ties and with the keys on chip: a lane loads four consecutive keys (one
+            // 128-bit load covers 128 keys per warp, i.e. four mask words), forms their keep bits
+            // as a nibble, and groups of eight lanes OR their shifted nibbles into one word.
+            const int nblk = (nwl + 3) / 4;
+            const bool nibble_path = !tie && keys_on_chip && (long long)nblk * 512 <= (long long)Ly.ring_bytes;
+            if (nibble_path) {
+                const uint4 *u4 = reinterpret_cast<const uint4 *>(ring);
+                for (int bk = warp; bk < nblk; bk += kWarps) {
+                    const int i0 = bk * 128 + 4 * lane;
+                    const uint4 x = u4[bk * 32 + lane];
+                    const unsigned uu[4] = {x.x, x.y, x.z, x.w};
+                    unsigned nib = 0u;
+#pragma unroll
+                    for (int j = 0; j < 4; ++j)
+                        if (i0 + j < n_local && (uu[j] & pmask) >= prefix) nib |= 1u << j;
+                    unsigned v = nib << (4 * (lane & 7));
+                    v |= __shfl_xor_sync(FULL, v, 1);
+                    v |= __shfl_xor_sync(FULL, v, 2);
+                    v |= __shfl_xor_sync(FULL, v, 4);
+                    const int wi = bk * 4 + (lane >> 3);
+                    if ((lane & 7) == 0 && wi < nwl) lmask[wi] = v;
                 }
-                const unsigned kb = __ballot_sync(FULL, keep);
-                if (lane == 0) lmask[wi] = kb;
+            }
+            // otherwise four words per warp per step: their keys are all loaded before the first ballot
+            for (int wi0 = warp; wi0 < (nibble_path ? 0 : nwl); wi0 += 4 * kWarps) {
+                unsigned uu[4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int i = (wi0 + j * kWarps) * 32 + lane;
+                    uu[j] = (wi0 + j * kWarps < nwl && i < n_local) ? uk[i] : 0u;
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const int wi = wi0 + j * kWarps;
+                    if (wi >= nwl) break;  // uniform over the warp
+                    const int i = wi * 32 + lane;
+                    const bool in = i < n_local;
+                    const unsigned u = uu[j];
+                    const bool gt = in && (u & pmask) > prefix;
+                    const bool eq = in && (u & pmask) == prefix;
+                    bool keep = gt || (eq && !tie);
+                    if (tie) {
+                        const unsigned eb = __ballot_sync(FULL, eq);
+                        const int rank = tie_off + tw[wi] + __popc(eb & ((1u << lane) - 1u));
+                        keep = gt || (eq && rank < need);
+                    }
+                    const unsigned kb = __ballot_sync(FULL, keep);
+                    if (lane == 0) lmask[wi] = kb;
+                }
             }
             cluster.sync();
             // global mask and its word prefix (identical in all CTAs)
@@ -1184,10 +1282,12 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                 __syncthreads();
             }
         }
-        // the next unit reuses this CTA's exchange buffers and masks: nobody may still be
-        // reading them
-        cluster.sync();
+        // No cluster barrier here: the buffers other CTAs read (the exchange record, the
+        // histograms, the mask words) are next written after the next unit's moments barrier,
+        // which a CTA reaches only after its own reads of this unit's values.
     }
+    // a CTA's shared memory must outlive every remote read of it
+    cluster.sync();
 
     // ---- the last CTA to finish publishes the new lengths ------------------------------
     if (a.mode == kModePrune && a.lens_out) {
