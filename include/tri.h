@@ -40,11 +40,17 @@
  *                       before any unit of the call is touched, so every unit of the
  *                       sequence is left untouched and lens_out[s] = lens[s].
  *       unit-level      a bounded wait that ran out, or a selection that did not give
- *                       exactly min(len, B) keys. Only that unit is left uncompacted; the
+ *                       exactly min(len, B) keys. That unit is left uncompacted; the
  *                       sequence's other units are pruned and lens_out[s] = min(len, B), so
  *                       the uncompacted unit then holds its first min(len, B) original rows
  *                       (a consistent cache, ascending positions, but not the method's
- *                       choice of keys). tri_get_failed_units lists such units.
+ *                       choice of keys). A group of CTAs whose wait ran out no longer trusts
+ *                       its copy pipeline: in the CUDA-core pass it also refuses the one unit
+ *                       it had already taken and takes no more (units are handed out
+ *                       dynamically, so other groups process the rest); in the pass over
+ *                       precomputed scores (max over offsets, tensor-core engine) units are
+ *                       assigned round robin and it refuses all its later units.
+ *                       tri_get_failed_units lists every such unit.
  *   - A context is bound to one device and is not thread-safe: serialise calls
  *     that share a context. Calls that share a context but run on different
  *     streams must not overlap on the GPU (they share the status word, the

@@ -461,6 +461,7 @@ tri::Args base_args(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budg
     a.mode = mode;
     a.status = c->d_status;
     a.counter = c->d_counter;
+    a.unit_next = c->d_counter + 1;
     a.seq_bad = seq_bad;
     a.wait_tries = c->wait_tries;
     a.inject_unit = c->inject_unit;
@@ -531,6 +532,10 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     a.unit_fail = pre.unit_fail;
     a.unit_base = unit_base;
     a.stagger = 1;
+    // the scoring variant hands units out dynamically from this counter, which the validation
+    // kernel launched just before zeroes; the precomputed-scores variant (one launch per chunk
+    // of layers) assigns them round robin
+    if (is_pre) a.unit_next = nullptr;
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
@@ -538,13 +543,16 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G, is_pre));
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)plan.cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // a programmatic dependent of the validation kernel launched just before on this stream
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     ce = cudaLaunchKernelEx(&cfg, fn, a);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx");
     return TRI_OK;
@@ -909,13 +917,16 @@ tri_status run_noalloc(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t b
     cfg.blockDim = dim3((unsigned)tri::cta_threads(c->G));
     cfg.dynamicSmemBytes = plan.smem;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)plan.cs;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    // a programmatic dependent of the validation kernel launched just before on this stream
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     ce = cudaLaunchKernelEx(&cfg, fn, a);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaLaunchKernelEx");
     return TRI_OK;
@@ -1078,14 +1089,14 @@ tri_status tri_create(tri_ctx **out, int device) {
     c->sm_count = p.multiProcessorCount;
     c->max_smem_optin = (int)p.sharedMemPerBlockOptin;
     if (cudaMalloc(&c->d_status, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMalloc(&c->d_counter, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMalloc(&c->d_counter, 2 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_count, sizeof(unsigned)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_units, sizeof(int32_t) * kFailCap) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ENOMEM;
     }
     if (cudaMemset(c->d_status, 0, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMemset(c->d_counter, 0, sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(c->d_counter, 0, 2 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMemset(c->d_fail_count, 0, sizeof(unsigned)) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ECUDA;

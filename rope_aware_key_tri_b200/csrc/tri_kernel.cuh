@@ -95,6 +95,8 @@ struct Args {
     long long slot_floats;       // floats per slot
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
+    unsigned int *unit_next;     // dynamic unit assignment: next free unit (null: round robin);
+                                 // zeroed by the validation kernel launched before
     int32_t *seq_bad;            // [batch] the validation kernel's verdicts (0: accepted)
     const float *pre;            // precomputed scores [n_units][cap_u][G] (tensor-core engine)
     const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing
@@ -114,9 +116,8 @@ struct Xch {
     float mn[8];
     float mx[8];
     int ties;
-    int kept;
     int fail;
-    int pad;
+    int next[2];  // rank 0: the cluster's next units under dynamic assignment (by parity)
 };
 
 struct Layout {
@@ -265,6 +266,18 @@ __device__ __noinline__ void stagger_wait(int n_units, int n_clusters, int cid, 
     for (int it = 0; it < (1 << 22) && global_ns() - t0 < wait_ns; ++it) __nanosleep(256);
 }
 
+// An int in cluster rank 0's shared memory at the address of *local (this CTA's copy of the
+// same variable). Written as asm so that the remote address is formed where it is used, not
+// held in registers across a loop.
+__device__ __forceinline__ int ld_rank0_int(const int *local) {
+    const unsigned laddr = (unsigned)__cvta_generic_to_shared(local);
+    unsigned raddr;
+    int v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, 0;" : "=r"(raddr) : "r"(laddr));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(raddr) : "memory");
+    return v;
+}
+
 __device__ __forceinline__ void prefetch_l1(const void *p) {
     asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
@@ -395,6 +408,10 @@ __device__ int block_exclusive_scan(int *a, int n, int *scratch /* kWarps + 2 in
 constexpr int kValidateThreads = 256;
 
 __global__ void __launch_bounds__(kValidateThreads) tri_validate_kernel(const Args a) {
+    // the fused kernel may be launched now: it waits for this grid's completion (and memory)
+    // before it reads a verdict or takes a unit
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (blockIdx.x == 0 && threadIdx.x == 0 && a.unit_next) *a.unit_next = 0u;
     const int s = blockIdx.x;
     const int N = __ldg(a.lens + s);
     const int n_layers = a.n_units / (a.batch * a.n_kv);
@@ -564,7 +581,8 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     // this cluster's scratch slot: scores [cap_u][G], then order keys [cap_u]
     float *sc = a.scratch + (long long)cid * a.slot_floats;
     unsigned *ukey = reinterpret_cast<unsigned *>(sc + (long long)a.cap_u * G);
-    const uint64_t pol_first = policy_evict_first();
+    // (the key stream's evict-first policy is created where a copy is issued: one lane per warp
+    // uses it, and a 64-bit register held by every lane would crowd the scoring loop)
     const uint64_t pol_last = policy_evict_last();
 
     // per-warp TMA buffers; the counters run on across units so that slot and phase
@@ -600,7 +618,6 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     const int tries = a.wait_tries;  // the drain after a timed-out wait
     // set once a bounded wait of this cluster ran out: the ring's barrier phases can no longer
     // be trusted, so the cluster refuses its remaining units instead of streaming them
-    bool dead = false;
     // Staggered start. With n_units = q n_clusters + r (0 < r), clusters r.. hold one unit fewer
     // and would idle at the end; they start about half a unit period late instead. Every
     // cluster then meets the memory-bound phases (key stream, compaction) at a different time
@@ -609,7 +626,70 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     // this cluster's first unit: its algorithmic bytes over the grid's share of 4.6 TB/s.
     if (a.stagger && a.mode == kModePrune && !PRE)
         stagger_wait(a.n_units, n_clusters, cid, a.lens, a.n_kv, a.batch, a.cap_u, a.budget, D);
-    for (int unit = cid; unit < a.n_units; unit += n_clusters) {
+    // Launched as a programmatic dependent of the validation kernel: everything above overlaps
+    // it; the verdicts, the status word and the cache are read only after its completion.
+    // (Without a preceding primary grid this returns at once.)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
+    // Unit assignment. Round robin (unit = cid + k n_clusters) over precomputed scores, dynamic
+    // in the scoring variant (which the validation kernel, zeroing the counter, always precedes):
+    // rank 0 takes the cluster's next unit from a global counter just before the unit's moments
+    // barrier (where the atomic's latency hides in the wait), and every CTA reads it at the end
+    // of the unit; a unit without that barrier takes the next one before an extra barrier. A
+    // cluster that started late, or runs slow, then simply takes fewer units. The slot of `next`
+    // written in iteration it + 1 was last read at the end of iteration it - 1, before that CTA
+    // arrived at iteration it's barrier, so no value is overwritten before both CTAs read it.
+    auto needs_work = [&](int u) {
+        const int su = (u / a.n_kv) % a.batch;
+        const int Nu = __ldg(a.lens + su);
+        const bool badu = __ldg(a.seq_bad + su) != 0 || Nu < 0 || Nu > a.cap_u;
+        return !badu && Nu > 0 && (a.mode == kModeScore || Nu > a.budget);
+    };
+    // The loop carries nothing in registers (the unit, the iteration count and the cluster's
+    // failure flag live in shared memory): a register carried across the whole unit loop spills
+    // in the scoring loop, which runs at the register limit.
+    constexpr bool DYN = !PRE;
+    __shared__ int unit_s, it_s, dead_s;
+    if (tid == 0) {
+        it_s = 0;
+        dead_s = 0;
+        unit_s = cid;
+    }
+    if constexpr (DYN) {
+        if (crank == 0 && tid == 0) xch->next[0] = (int)atomicAdd(a.unit_next, 1u);
+        cluster.sync();
+        if (tid == 0) unit_s = ld_rank0_int(&xch->next[0]);
+    }
+    __syncthreads();
+    // the unit after this one, in every thread; two block barriers per unit
+    auto advance = [&]() {
+        __syncthreads();  // every thread has read this iteration's unit_s and it_s
+        if (tid == 0) {
+            int nxt;
+            if constexpr (!DYN) {
+                nxt = unit_s + n_clusters;
+            } else {
+                nxt = ld_rank0_int(&xch->next[(it_s + 1) & 1]);
+                if (dead_s) {
+                    // the unit already taken is refused like the one whose wait ran out; the
+                    // cluster takes no more, the other clusters process the rest
+                    if (nxt < a.n_units && needs_work(nxt) && crank == 0)
+                        record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
+                                            a.unit_base + nxt);
+                    nxt = a.n_units;
+                }
+            }
+            unit_s = nxt;
+            ++it_s;
+        }
+        __syncthreads();
+    };
+    auto take_next = [&]() {
+        if (DYN && crank == 0 && tid == 0) xch->next[(it_s + 1) & 1] = (int)atomicAdd(a.unit_next, 1u);
+    };
+    for (;; advance()) {
+        const int unit = unit_s;  // uniform
+        if (unit >= a.n_units) break;
         const int g = unit % a.n_kv;
         const int s = (unit / a.n_kv) % a.batch;
         const int lr = unit / (a.n_kv * a.batch);
@@ -619,7 +699,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
         // skipped whole; the capacity test is repeated here so that no access depends on it
         const bool bad = __ldg(a.seq_bad + s) != 0 || N < 0 || N > a.cap_u;
         const bool work0 = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
-        if (dead) {  // uniform over the cluster
+        if (!DYN && dead_s) {  // uniform over the cluster (a dynamic cluster stops instead)
             if (work0 && crank == 0 && tid == 0)
                 record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
                                     a.unit_base + unit);
@@ -630,7 +710,13 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
         if (missing && crank == 0 && tid == 0)
             record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout, a.unit_base + unit);
         const bool work = work0 && !missing;
-        if (!work) continue;  // uniform over the cluster: no cluster barrier is skipped unevenly
+        if (!work) {  // uniform over the cluster: no cluster barrier is skipped unevenly
+            if constexpr (DYN) {  // in place of the moments barrier (see above)
+                take_next();
+                cluster.sync();
+            }
+            continue;
+        }
 
         const int kpc = ((N + cs - 1) / cs + 31) / 32 * 32;
         const int begin = crank * kpc;
@@ -657,7 +743,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
             mbar_expect_tx(bar, (unsigned)nrows * D * 2u);
             if (withhold) return;
             tma_load_1d(ring + (size_t)(warp * nslot + slot) * kStageBytes, a.K + r * D,
-                        (unsigned)nrows * D * 2u, bar, pol_first);
+                        (unsigned)nrows * D * 2u, bar, policy_evict_first());
         };
         __syncthreads();  // the ring is free (previous unit's staging reads are done)
         {
@@ -894,6 +980,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
             }
             if (tid == 0) xch->fail = fail;
         }
+        take_next();
         cluster.sync();
         // every CTA gathers the cluster's partials (one remote load per thread, all in
         // flight together) and folds them in rank order
@@ -935,7 +1022,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                                     a.unit_base + unit);
         }
         __syncthreads();
-        dead = anyfail_s != 0;
+        if (tid == 0 && anyfail_s) dead_s = 1;  // read after the next block barrier
 
         // ---- z-score, max over the group, order key --------------------------------------
         // The order keys live in the (now idle) TMA ring when they fit, else in the scratch

@@ -105,7 +105,12 @@ def test_withheld_copy_times_out_and_leaves_units_uncompacted(combine):
     assert n_failed == len(failed) and victim in failed
     failed = sorted(set(failed))
     if combine == "mean":
-        # the cluster whose wait ran out refuses its later units: victim, victim + c, ... for its stride c
+        # units are handed out dynamically: the cluster whose wait ran out refuses the unit it had
+        # already taken next (when that one needs pruning) and takes no more
+        assert len(failed) <= 2, failed
+        assert all(lens0[cache.unit_index(u)[1]] > spec.budget for u in failed), failed
+    else:
+        # round robin over precomputed scores: the cluster refuses its later units, victim + k c
         if len(failed) > 1:
             c = int(np.gcd.reduce(np.diff(failed)))
             want = [u for u in range(victim, U, c)
