@@ -59,6 +59,7 @@ __host__ __device__ constexpr int mx_epi_groups(int acc_cols) { return 512 / acc
 __host__ __device__ constexpr int mx_threads_of(int acc_cols) { return 64 + 128 * mx_epi_groups(acc_cols); }
 constexpr int kMxTile = 128;       // keys per tile (the MMA's M)
 constexpr int kMxMaxStages = 6;
+constexpr int kMxMaxAcc = 6;       // accumulator buffers the barrier block has room for
 constexpr unsigned kMxChunkBytes = kMxTile * 128u;  // one 64-dim chunk of a tile: 128 rows x 128 B
 
 // Columns per head: the offset count padded to one of three compile-time counts (the padding
@@ -354,8 +355,9 @@ __host__ __device__ inline MxLayout mx_layout(int D, int G, int ncol, int nst) {
     L.stage = 0;
     L.image = (unsigned)nst * stage_bytes;
     L.bars = L.image + 2u * mx_image_bytes(D, G, ncol);
-    // full[nst], empty[nst], bfull[2], bempty[2], accfull[4], accempty[4], TMEM address, abort flag
-    L.total = L.bars + (unsigned)(2 * nst + 12) * 8u + 16u + 1024u;  // + alignment slack
+    // full[nst], empty[nst], bfull[2], bempty[2], accfull[kMxMaxAcc], accempty[kMxMaxAcc], TMEM
+    // address, abort flag
+    L.total = L.bars + (unsigned)(2 * nst + 4 + 2 * kMxMaxAcc) * 8u + 16u + 1024u;  // + alignment slack
     return L;
 }
 
@@ -380,6 +382,7 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
     constexpr int NCH = CAT ? 0 : (G * NOFF + 31) / 32;  // 32-column chunks of the max
     constexpr int REAL = G * NOFF;      // columns that hold a (head, offset) score
     static_assert(NACC % NE == 0 && NACC * ACC <= 512, "accumulator buffers");
+    static_assert(NACC <= kMxMaxAcc, "the barrier block holds kMxMaxAcc accumulator buffers");
     constexpr unsigned kStageBytes = KCH * kMxChunkBytes;
     extern __shared__ unsigned char mx_smem_raw[];
     unsigned char *smem = reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(mx_smem_raw) + 1023) &
@@ -393,8 +396,8 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
     uint64_t *bfull = empty + nst;
     uint64_t *bempty = bfull + 2;
     uint64_t *accfull = bempty + 2;
-    uint64_t *accempty = accfull + 4;
-    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + 4);
+    uint64_t *accempty = accfull + kMxMaxAcc;
+    uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accempty + kMxMaxAcc);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
