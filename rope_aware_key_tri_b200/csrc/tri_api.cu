@@ -532,10 +532,8 @@ tri_status launch_fused(tri_ctx *c, KernelFn fn, const tri_kv *kv, const int32_t
     a.unit_fail = pre.unit_fail;
     a.unit_base = unit_base;
     a.stagger = 1;
-    // the scoring variant hands units out dynamically from this counter, which the validation
-    // kernel launched just before zeroes; the precomputed-scores variant (one launch per chunk
-    // of layers) assigns them round robin
-    if (is_pre) a.unit_next = nullptr;
+    // units are handed out from a.unit_next (set by base_args), which the kernel launched just
+    // before zeroes: the validation kernel, or the tensor-core scoring kernel of this chunk
 
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
@@ -694,6 +692,7 @@ tri_status run_max(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budge
     m.seq_bad = c->d_seq_bad;
     m.wait_tries = c->wait_tries;
     m.inject_unit = c->inject_unit;
+    m.unit_next = c->d_counter + 1;
     cudaStream_t cs = static_cast<cudaStream_t>(stream);
 
     tri::tri_mx_prefix_kernel<<<1, 32, 0, cs>>>(m);

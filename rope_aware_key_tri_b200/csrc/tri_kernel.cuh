@@ -616,14 +616,11 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     const int Hq = a.n_kv * G;
 
     const int tries = a.wait_tries;  // the drain after a timed-out wait
-    // set once a bounded wait of this cluster ran out: the ring's barrier phases can no longer
-    // be trusted, so the cluster refuses its remaining units instead of streaming them
-    // Staggered start. With n_units = q n_clusters + r (0 < r), clusters r.. hold one unit fewer
-    // and would idle at the end; they start about half a unit period late instead. Every
-    // cluster then meets the memory-bound phases (key stream, compaction) at a different time
-    // from the latency-bound ones (z-score, select, mask) of a fifth of the grid, where all
-    // clusters would otherwise reach each kind of phase together. The period is estimated from
-    // this cluster's first unit: its algorithmic bytes over the grid's share of 4.6 TB/s.
+    // Staggered start. With n_units = q n_clusters + r (0 < r), an even split leaves clusters
+    // r.. one unit short, idle at the end; they start about half a unit period late instead.
+    // The grid's clusters then no longer reach the memory-bound phases (key stream, compaction)
+    // and the latency-bound ones (z-score, select, mask) all at the same time. The period is
+    // estimated from unit cid: its algorithmic bytes over the grid's share of 4.6 TB/s.
     if (a.stagger && a.mode == kModePrune && !PRE)
         stagger_wait(a.n_units, n_clusters, cid, a.lens, a.n_kv, a.batch, a.cap_u, a.budget, D);
     // Launched as a programmatic dependent of the validation kernel: everything above overlaps
@@ -631,12 +628,13 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     // (Without a preceding primary grid this returns at once.)
     asm volatile("griddepcontrol.wait;" ::: "memory");
 
-    // Unit assignment. Round robin (unit = cid + k n_clusters) over precomputed scores, dynamic
-    // in the scoring variant (which the validation kernel, zeroing the counter, always precedes):
-    // rank 0 takes the cluster's next unit from a global counter just before the unit's moments
-    // barrier (where the atomic's latency hides in the wait), and every CTA reads it at the end
-    // of the unit; a unit without that barrier takes the next one before an extra barrier. A
-    // cluster that started late, or runs slow, then simply takes fewer units. The slot of `next`
+    // Dynamic unit assignment. The kernel launched just before (the validation kernel, or the
+    // tensor-core scoring kernel before the precomputed-scores variant) zeroes the counter a.unit_next.
+    // Rank 0 takes the cluster's next unit from it just before the unit's moments barrier (where
+    // the atomic's latency hides in the wait), and every CTA reads it at the end of the unit; a
+    // unit without that barrier takes the next one before an extra barrier. A cluster that
+    // started late (placed after other grids' blocks left) or runs slow simply takes fewer units,
+    // and ragged units balance over the clusters. The slot of `next`
     // written in iteration it + 1 was last read at the end of iteration it - 1, before that CTA
     // arrived at iteration it's barrier, so no value is overwritten before both CTAs read it.
     auto needs_work = [&](int u) {
@@ -648,36 +646,27 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
     // The loop carries nothing in registers (the unit, the iteration count and the cluster's
     // failure flag live in shared memory): a register carried across the whole unit loop spills
     // in the scoring loop, which runs at the register limit.
-    constexpr bool DYN = !PRE;
     __shared__ int unit_s, it_s, dead_s;
     if (tid == 0) {
         it_s = 0;
         dead_s = 0;
-        unit_s = cid;
     }
-    if constexpr (DYN) {
-        if (crank == 0 && tid == 0) xch->next[0] = (int)atomicAdd(a.unit_next, 1u);
-        cluster.sync();
-        if (tid == 0) unit_s = ld_rank0_int(&xch->next[0]);
-    }
+    if (crank == 0 && tid == 0) xch->next[0] = (int)atomicAdd(a.unit_next, 1u);
+    cluster.sync();
+    if (tid == 0) unit_s = ld_rank0_int(&xch->next[0]);
     __syncthreads();
     // the unit after this one, in every thread; two block barriers per unit
     auto advance = [&]() {
         __syncthreads();  // every thread has read this iteration's unit_s and it_s
         if (tid == 0) {
-            int nxt;
-            if constexpr (!DYN) {
-                nxt = unit_s + n_clusters;
-            } else {
-                nxt = ld_rank0_int(&xch->next[(it_s + 1) & 1]);
-                if (dead_s) {
-                    // the unit already taken is refused like the one whose wait ran out; the
-                    // cluster takes no more, the other clusters process the rest
-                    if (nxt < a.n_units && needs_work(nxt) && crank == 0)
-                        record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
-                                            a.unit_base + nxt);
-                    nxt = a.n_units;
-                }
+            int nxt = ld_rank0_int(&xch->next[(it_s + 1) & 1]);
+            if (dead_s) {
+                // the unit already taken is refused like the one whose wait ran out; the
+                // cluster takes no more, the other clusters process the rest
+                if (nxt < a.n_units && needs_work(nxt) && crank == 0)
+                    record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
+                                        a.unit_base + nxt);
+                nxt = a.n_units;
             }
             unit_s = nxt;
             ++it_s;
@@ -685,7 +674,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
         __syncthreads();
     };
     auto take_next = [&]() {
-        if (DYN && crank == 0 && tid == 0) xch->next[(it_s + 1) & 1] = (int)atomicAdd(a.unit_next, 1u);
+        if (crank == 0 && tid == 0) xch->next[(it_s + 1) & 1] = (int)atomicAdd(a.unit_next, 1u);
     };
     for (;; advance()) {
         const int unit = unit_s;  // uniform
@@ -699,22 +688,14 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
         // skipped whole; the capacity test is repeated here so that no access depends on it
         const bool bad = __ldg(a.seq_bad + s) != 0 || N < 0 || N > a.cap_u;
         const bool work0 = !bad && N > 0 && (a.mode == kModeScore || N > a.budget);
-        if (!DYN && dead_s) {  // uniform over the cluster (a dynamic cluster stops instead)
-            if (work0 && crank == 0 && tid == 0)
-                record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout,
-                                    a.unit_base + unit);
-            continue;
-        }
         bool missing = false;  // the scoring kernel gave up on this unit (it recorded why)
         if constexpr (PRE) missing = work0 && __ldg(a.unit_fail + unit) != 0;
         if (missing && crank == 0 && tid == 0)
             record_unit_failure(a.status, a.fail_count, a.fail_units, a.fail_cap, kDevTimeout, a.unit_base + unit);
         const bool work = work0 && !missing;
         if (!work) {  // uniform over the cluster: no cluster barrier is skipped unevenly
-            if constexpr (DYN) {  // in place of the moments barrier (see above)
-                take_next();
-                cluster.sync();
-            }
+            take_next();  // and the barrier in place of the moments barrier (see above)
+            cluster.sync();
             continue;
         }
 

@@ -115,6 +115,7 @@ struct MxArgs {
     const int32_t *seq_bad;      // [batch] sequences refused by the validation kernel (no tiles)
     int wait_tries;              // tries (about 1 ms each) of every bounded wait
     long long inject_unit;       // test hook: the unit whose first key tile is withheld (-1: none)
+    unsigned *unit_next;         // the fused kernel's unit counter, zeroed here for the launch after
 };
 
 // ---------------------------------------------------------------------------------
@@ -401,6 +402,10 @@ __global__ void __launch_bounds__(mx_threads(G, NOFF), 1) tri_mx_score_kernel(co
     volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_holder + 1);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    // the fused select/compaction over these scores may be launched now (it waits for this grid's
+    // completion before it reads a score or takes a unit); its unit counter starts from zero
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    if (blockIdx.x == 0 && tid == 0) *a.unit_next = 0u;
 
     // this CTA's tile range
     const int per_layer = __ldg(a.tile_prefix + a.batch);
