@@ -45,11 +45,11 @@
  *                       the uncompacted unit then holds its first min(len, B) original rows
  *                       (a consistent cache, ascending positions, but not the method's
  *                       choice of keys). A group of CTAs whose wait ran out no longer trusts
- *                       its copy pipeline: in the CUDA-core pass it also refuses the one unit
- *                       it had already taken and takes no more (units are handed out
- *                       dynamically, so other groups process the rest); in the pass over
- *                       precomputed scores (max over offsets, tensor-core engine) units are
- *                       assigned round robin and it refuses all its later units.
+ *                       its copy pipeline: it also refuses the one unit it had already taken
+ *                       and takes no more (units are handed out dynamically, so other groups
+ *                       process the rest). In the tensor-core scoring kernel (max over
+ *                       offsets, tensor-core engine) a wait that ran out ends that CTA's tile
+ *                       range, and every unit the range touches is refused.
  *                       tri_get_failed_units lists every such unit.
  *   - A context is bound to one device and is not thread-safe: serialise calls
  *     that share a context. Calls that share a context but run on different

@@ -95,8 +95,8 @@ struct Args {
     long long slot_floats;       // floats per slot
     unsigned long long *status;  // first device-detected problem
     unsigned int *counter;       // completed-CTA counter (last CTA updates lens_out)
-    unsigned int *unit_next;     // dynamic unit assignment: next free unit (null: round robin);
-                                 // zeroed by the validation kernel launched before
+    unsigned int *unit_next;     // dynamic unit assignment: the next free unit; zeroed by the
+                                 // kernel launched just before (validation or tensor-core scoring)
     int32_t *seq_bad;            // [batch] the validation kernel's verdicts (0: accepted)
     const float *pre;            // precomputed scores [n_units][cap_u][G] (tensor-core engine)
     const int32_t *unit_fail;    // [n_units] units whose precomputed scores are missing

@@ -110,7 +110,7 @@ def test_withheld_copy_times_out_and_leaves_units_uncompacted(combine):
         assert len(failed) <= 2, failed
         assert all(lens0[cache.unit_index(u)[1]] > spec.budget for u in failed), failed
     else:
-        # round robin over precomputed scores: the cluster refuses its later units, victim + k c
+        # the tensor-core scoring kernel refuses the units of the tile range it abandoned
         if len(failed) > 1:
             c = int(np.gcd.reduce(np.diff(failed)))
             want = [u for u in range(victim, U, c)
