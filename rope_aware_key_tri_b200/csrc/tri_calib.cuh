@@ -15,10 +15,13 @@
 // The pass is one stream over Q (HBM-bound): a CTA takes a fixed chunk of tokens of one
 // layer and 128 threads; each thread owns 4 bands of one head (16 bytes per token: two 8-byte
 // pieces in the half layout, where a band's two dims sit d/2 apart, one 16-byte piece in the
-// interleaved layout), sums re, im in fp64 and |q_f| (from the exact bf16 components: one
-// fp32 rounding of re^2 + im^2, a correctly rounded fp32 square root) in fp64, and writes its
-// chunk's sums; 8 tokens are loaded before any is used. A second launch adds the chunks in
-// order, so the result does not depend on the GPU, and forms the means and R.
+// interleaved layout), sums re, im and |q_f| (from the exact bf16 components: one fp32
+// rounding of re^2 + im^2, a correctly rounded fp32 square root) over the chunk, and writes its
+// chunk's sums; 8 tokens are loaded before any is used, added in fp32 (re and im as one packed
+// pair), and each 8-token partial is added to fp64 chunk sums. A partial of 8 values is off by
+// at most 7 * 2^-24 of the sum of their magnitudes (4.2e-7); the fp64 sums add nothing
+// measurable. A second launch adds the chunks in order, so the result does not depend on the
+// GPU, and forms the means and R.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -59,7 +62,9 @@ __global__ void __launch_bounds__(kCalThreads, kCalMinBlocks) tri_calib_partial_
     double sr[NB], si[NB], sm[NB];
 #pragma unroll
     for (int k = 0; k < NB; ++k) sr[k] = si[k] = sm[k] = 0.0;
-    // one token's pieces (four 32-bit words: 4 bands) into the band sums
+    float2 pri[NB];  // fp32 partials of the current batch: (re, im) and |q_f|
+    float pm[NB];
+    // one token's pieces (four 32-bit words: 4 bands) into the batch partials
     auto add = [&](uint4 w) {
         const unsigned wv[4] = {w.x, w.y, w.z, w.w};
         float re[NB], im[NB];
@@ -81,9 +86,23 @@ __global__ void __launch_bounds__(kCalThreads, kCalMinBlocks) tri_calib_partial_
         }
 #pragma unroll
         for (int k = 0; k < NB; ++k) {
-            sr[k] += (double)re[k];
-            si[k] += (double)im[k];
-            sm[k] += (double)__fsqrt_rn(fmaf(re[k], re[k], im[k] * im[k]));
+            pri[k] = __fadd2_rn(pri[k], make_float2(re[k], im[k]));
+            pm[k] += __fsqrt_rn(fmaf(re[k], re[k], im[k] * im[k]));
+        }
+    };
+    auto clear = [&]() {
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+            pri[k] = make_float2(0.f, 0.f);
+            pm[k] = 0.f;
+        }
+    };
+    auto flush = [&]() {
+#pragma unroll
+        for (int k = 0; k < NB; ++k) {
+            sr[k] += (double)pri[k].x;
+            si[k] += (double)pri[k].y;
+            sm[k] += (double)pm[k];
         }
     };
     auto load = [&](int t) {
@@ -101,10 +120,15 @@ __global__ void __launch_bounds__(kCalThreads, kCalMinBlocks) tri_calib_partial_
         uint4 v[kCalUnroll];
 #pragma unroll
         for (int u = 0; u < kCalUnroll; ++u) v[u] = load(t + u);
+        clear();
 #pragma unroll
         for (int u = 0; u < kCalUnroll; ++u) add(v[u]);
+        flush();
     }
-    for (; t < t1; ++t) add(load(t));  // the chunk's ragged tail (the last chunk of a layer only)
+    // the chunk's ragged tail (the last chunk of a layer only): fewer than 8 tokens, one partial
+    clear();
+    for (; t < t1; ++t) add(load(t));
+    flush();
     double *p = part + ((((size_t)chunk * L + l) * Hq + h) * F + (size_t)slot * NB) * 3;
 #pragma unroll
     for (int k = 0; k < NB; ++k) {

@@ -2,10 +2,12 @@
 
 Seeded query samples (tri_synth.make_queries: per-head centres with spreads from tight to
 diffuse, one all-zero band) are reduced on the GPU and by the oracle on the same bits.
-Tolerances: the GPU sums in fp64 but takes |q_f| with one fp32 rounding of re^2 + im^2 and a
-correctly rounded fp32 square root (relative error below 1.2e-7 per sample), and rounds the
-outputs to fp32 once. So E|q_f| must agree to 1e-6 relative, the centre to 1e-6 of E|q_f|
-(it may be near zero), and R (in [0, 1]) to 2e-6 absolute. An all-zero band gives exactly 0.
+Tolerances: the GPU takes |q_f| with one fp32 rounding of re^2 + im^2 and a correctly rounded
+fp32 square root (relative error below 1.2e-7 per sample), adds 8 tokens at a time in fp32 (at
+most 7 * 2^-24 = 4.2e-7 of the sum of the magnitudes added), adds those partials in fp64, and
+rounds the outputs to fp32 once (6e-8). So E|q_f| must agree to 1e-6 relative, the centre to
+1e-6 of E|q_f| (it may be near zero; re and im are each bounded by |q_f|), and R (in [0, 1]) to
+2e-6 absolute. An all-zero band gives exactly 0.
 """
 import numpy as np
 import pytest
