@@ -59,6 +59,7 @@ struct tri_ctx {
     size_t att_part_bytes = 0;
     // device bookkeeping
     unsigned long long *d_status = nullptr;
+    // [0] CTAs of the fused kernel done, [1] its next free unit, [2] CTAs of tri_append done
     unsigned int *d_counter = nullptr;
     int32_t *d_seq_bad = nullptr;    // per-sequence verdict of the validation kernel
     int seq_bad_cap = 0;
@@ -455,6 +456,10 @@ tri::Args base_args(tri_ctx *c, const tri_kv *kv, const int32_t *t, int32_t budg
     a.page_size = paged ? kv->page_size : 0;
     a.max_pages = paged ? kv->max_pages : 0;
     a.n_pages = paged ? kv->n_pages : 0;
+    a.page_shift = -1;
+    if (paged && (kv->page_size & (kv->page_size - 1)) == 0)
+        for (int b = 0; (1 << b) <= kv->page_size; ++b)
+            if ((1 << b) == kv->page_size) a.page_shift = b;
     a.layer_begin = kv->layer_begin;
     a.budget = mode == tri::kModePrune ? budget : 0x7fffffff;
     a.n_units = (int)((long long)kv->n_layers * kv->batch * c->Hkv);
@@ -1088,14 +1093,14 @@ tri_status tri_create(tri_ctx **out, int device) {
     c->sm_count = p.multiProcessorCount;
     c->max_smem_optin = (int)p.sharedMemPerBlockOptin;
     if (cudaMalloc(&c->d_status, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMalloc(&c->d_counter, 2 * sizeof(unsigned int)) != cudaSuccess ||
+        cudaMalloc(&c->d_counter, 3 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_count, sizeof(unsigned)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_units, sizeof(int32_t) * kFailCap) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ENOMEM;
     }
     if (cudaMemset(c->d_status, 0, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMemset(c->d_counter, 0, 2 * sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(c->d_counter, 0, 3 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMemset(c->d_fail_count, 0, sizeof(unsigned)) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ECUDA;
@@ -1301,6 +1306,8 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     a.n_pages = kv->n_pages;
     a.status = c->d_status;
     a.seq_bad = c->d_append_bad;
+    a.lens_out = kv->lens_out;
+    a.done = c->d_counter + 2;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
     if (c->D == 128)
@@ -1309,10 +1316,6 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
         tri::tri_append_kernel<64><<<blocks, tri::kAppendWarps * 32, 0, st>>>(a);
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append rows");
-    tri::tri_append_lens_kernel<<<(unsigned)((kv->batch + 255) / 256), 256, 0, st>>>(kv->lens, kv->lens_out,
-                                                                                       c->d_append_bad, kv->batch);
-    ce = cudaGetLastError();
-    if (ce != cudaSuccess) return cuda_fail(c, ce, "append lengths");
     return TRI_OK;
 }
 

@@ -78,6 +78,7 @@ struct Args {
     const int32_t *t;
     int batch, n_kv, cap_u;
     int paged, page_size, max_pages, n_pages;
+    int page_shift;              // log2(page_size) when a power of two, else -1
     int layer_begin;
     int budget;
     int n_units;
@@ -327,8 +328,17 @@ __device__ __forceinline__ void record_unit_failure(unsigned long long *st, unsi
 // Row index (in rows of head_dim elements) of logical slot i of a unit.
 __device__ __forceinline__ long long row_of(const Args &a, int lr, int s, int g, int i) {
     if (!a.paged) return (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + i;
-    const int page = __ldg(a.block_table + (long long)s * a.max_pages + i / a.page_size);
-    return (((long long)lr * a.n_pages + page) * a.n_kv + g) * (long long)a.page_size + (i % a.page_size);
+    // a row address per moved row and lane: shifts for the usual power-of-two page sizes
+    int pi, po;
+    if (a.page_shift >= 0) {
+        pi = i >> a.page_shift;
+        po = i & (a.page_size - 1);
+    } else {
+        pi = i / a.page_size;
+        po = i - pi * a.page_size;
+    }
+    const int page = __ldg(a.block_table + (long long)s * a.max_pages + pi);
+    return (((long long)lr * a.n_pages + page) * a.n_kv + g) * (long long)a.page_size + po;
 }
 
 // k-th (0-based) set bit of m.
