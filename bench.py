@@ -540,7 +540,7 @@ def run_calibrate(args):
     nbytes = q.numel() * 2 + sum(x.numel() * 4 for x in out)
     res = {"metric": CAL_METRIC, "value": rows / (ms * 1e-3), "unit": "rows/s", "n_gpus": 1,
            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp64 sums", "data": "synthetic",
+           "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in, fp32 8-token partials, fp64 sums", "data": "synthetic",
            "config": {"workload": "qwen3_8b_calibration_10k", "layers": L, "tokens": T, "q_heads": Hq,
                       "head_dim": d, "layout": "half",
                       "timed": "CUDA events around tri_calibrate_estimate (partial sums + means)"},
