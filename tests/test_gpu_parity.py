@@ -312,3 +312,38 @@ def test_host_validation_with_device():
     # nothing above launched anything: the cache is unchanged
     assert cache.lens_host.tolist() == [256]
     gu_ctx.close(); ctx.close()
+
+
+@pytest.mark.parametrize("paged", [False, True])
+def test_prune_captured_in_cuda_graph_equals_eager(paged):
+    """tri_prune's two launches (the validation kernel, then the fused kernel as its programmatic
+    dependent, taking units from a counter the validation zeroes) captured in a CUDA graph and
+    replayed give the same cache, bit for bit, as the same call issued directly. Four layers of
+    the single-layer decode workload: 512 units, several per cluster."""
+    spec = ts.replace(ts.WORKLOADS["qwen3_8b_decode_b16_2176"], n_layers=4,
+                      page_size=64 if paged else 0)
+    base = ts.make_cache(spec, 41).to("cuda")
+    eager, captured = base.clone(), base.clone()
+    ctx = gu.context_for(base)
+    # the eager call also sizes the context's scratch and caches the launch plan, so the captured
+    # call allocates nothing
+    assert gu.gpu_prune(ctx, eager)[0] == tri.TRI_OK
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=side, capture_error_mode="relaxed"):
+        ctx.prune(captured.K, captured.V, captured.pos, captured.lens, captured.t, spec.budget,
+                  block_table=captured.block_table)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    assert torch.equal(captured.lens, base.lens)  # capturing ran nothing
+    g.replay()
+    torch.cuda.synchronize()
+    assert ctx.get_error()[0] == tri.TRI_OK
+    assert torch.equal(eager.lens, captured.lens)
+    assert eager.lens_host.tolist() == [spec.budget] * spec.batch
+    assert torch.equal(eager.K.view(torch.int16), captured.K.view(torch.int16))
+    assert torch.equal(eager.V.view(torch.int16), captured.V.view(torch.int16))
+    assert torch.equal(eager.pos, captured.pos)
+    del g
+    ctx.close()
