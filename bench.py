@@ -638,8 +638,7 @@ def run_decode(args):
                 for s in range(batch):
                     bt[s, host_len // ps] = free.pop(0)
                 bt_dev.copy_(torch.from_numpy(bt))  # from pageable memory: the host waits for it
-            ctx.append(K, V, P, lens, bt_dev, new_k[i], new_v[i], tpos)
-            tpos.add_(1)
+            ctx.append(K, V, P, lens, bt_dev, new_k[i], new_v[i], tpos, advance=True)
             host_len += 1
         ctx.prune(K, V, P, lens, tpos, B, block_table=bt_dev)
         host_len = B
@@ -678,8 +677,7 @@ def run_decode(args):
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=side, capture_error_mode="relaxed"):
                 for i in range(half * ps, (half + 1) * ps):
-                    ctx.append(K, V, P, lens, bt_dev, new_k[i], new_v[i], tpos)
-                    tpos.add_(1)
+                    ctx.append(K, V, P, lens, bt_dev, new_k[i], new_v[i], tpos, advance=True)
             graphs.append(gr)
         stream.wait_stream(side)
         torch.cuda.synchronize()
@@ -734,7 +732,7 @@ def run_decode(args):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": "qwen3_8b_periodic_36l_3200 (paged, 64-token pages)", "layers": L,
                        "kv_heads": Hkv, "group": G, "head_dim": d, "batch": batch, "budget": B, "cadence": cad,
-                       "timed": "CUDA events around one cycle: 128 tri_append (two CUDA-graph replays) + "
+                       "timed": "CUDA events around one cycle: 128 tri_append_advance (two CUDA-graph replays) + "
                                 "block-table copies (pinned, asynchronous) + tri_prune"},
             "roofline": roofline_hbm(nbytes, ms),
             # 128 appends of one launch each, the prune's validation and fused kernels

@@ -197,6 +197,17 @@ TRI_API tri_status tri_append(tri_ctx *ctx, const tri_kv *kv, const void *K_new,
                               const int32_t *pos_new, void *stream);
 
 /*
+ * tri_append for a decode loop whose next token position follows the last one: the same append
+ * of the rows and of the position pos[s], after which pos[s] += 1 for every sequence that
+ * accepted the token (a refused sequence keeps its position as it keeps its length). The
+ * caller's per-step position update is thereby part of the same single launch.
+ *   pos      int32 [batch] device: in, the new token's positions; out, the next ones
+ * Everything else as tri_append.
+ */
+TRI_API tri_status tri_append_advance(tri_ctx *ctx, const tri_kv *kv, const void *K_new, const void *V_new,
+                                      int32_t *pos, void *stream);
+
+/*
  * Estimate the calibration statistics from pre-RoPE query samples (the pages' offline
  * calibration step: [Deep-dive] §3.4; the statistics of [Stage] §TriAttention：把理论变成算法
  * items 1-2 and the concentration of [Stage] §破局之道, taken per band).

@@ -1264,9 +1264,9 @@ tri_status tri_calibrate_estimate(tri_ctx *c, const void *Q, int n_layers, int T
     return TRI_OK;
 }
 
-tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, const int32_t *pos_new,
-                      void *stream) {
-    NvtxRange r("tri_append");
+namespace {
+tri_status append_impl(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, const int32_t *pos_new,
+                       bool advance, void *stream) {
     if (!c || !kv || !K_new || !V_new || !pos_new) return TRI_EINVAL;
     if (!c->loaded) return TRI_ESTATE;
     if (c->D != 64 && c->D != 128) return TRI_EUNSUPPORTED;
@@ -1308,6 +1308,7 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     a.seq_bad = c->d_append_bad;
     a.lens_out = kv->lens_out;
     a.done = c->d_counter + 2;
+    a.pos_adv = advance ? const_cast<int32_t *>(pos_new) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
     if (c->D == 128)
@@ -1317,6 +1318,19 @@ tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const voi
     ce = cudaGetLastError();
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append rows");
     return TRI_OK;
+}
+}  // namespace
+
+tri_status tri_append(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, const int32_t *pos_new,
+                      void *stream) {
+    NvtxRange r("tri_append");
+    return append_impl(c, kv, K_new, V_new, pos_new, false, stream);
+}
+
+tri_status tri_append_advance(tri_ctx *c, const tri_kv *kv, const void *K_new, const void *V_new, int32_t *pos,
+                              void *stream) {
+    NvtxRange r("tri_append_advance");
+    return append_impl(c, kv, K_new, V_new, pos, true, stream);
 }
 
 tri_status tri_set_offset_combine(tri_ctx *c, int combine) {

@@ -30,6 +30,7 @@ struct AppendArgs {
     unsigned long long *status;   // first device-detected problem
     int32_t *seq_bad;             // [batch] refused sequences
     unsigned *done;               // completed-CTA counter (zero between launches)
+    int32_t *pos_adv;             // pos_new itself, advanced by one for the accepted sequences (or null)
 };
 
 __device__ __forceinline__ void append_record(unsigned long long *st, int code, long long unit) {
@@ -76,9 +77,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32) tri_append_kernel(const App
             if (lane == 0) a.pos[row] = __ldg(a.pos_new + s);
         }
     }
-    // lens_out[s] = lens[s] + 1 for every sequence whose rows all went in; refused sequences
-    // keep their length and their flag is cleared for the next call. Done by the last CTA to
-    // finish, after every CTA has read the lengths and raised its flags.
+    // lens_out[s] = lens[s] + 1 for every sequence whose rows all went in (and, when asked, its
+    // next position pos_new[s] + 1); refused sequences keep both and their flag is cleared for
+    // the next call. Done by the last CTA to finish, after every CTA has read the lengths and
+    // positions and raised its flags.
     __shared__ int last_s;
     __syncthreads();
     if (threadIdx.x == 0) {
@@ -92,6 +94,7 @@ __global__ void __launch_bounds__(kAppendWarps * 32) tri_append_kernel(const App
             const int n = a.lens[s];
             const int refused = atomicExch(a.seq_bad + s, 0);
             a.lens_out[s] = refused ? n : n + 1;
+            if (a.pos_adv && !refused) a.pos_adv[s] += 1;  // the next token's position
         }
         if (threadIdx.x == 0) atomicExch(a.done, 0u);
     }

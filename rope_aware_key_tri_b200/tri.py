@@ -67,6 +67,7 @@ def _load():
     L.tri_calibrate_estimate.argtypes = [P, P, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                          ctypes.c_int, P, P, P, P]
     L.tri_append.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
+    L.tri_append_advance.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P, P]
     L.tri_get_error.argtypes = [P, P, ctypes.POINTER(I32), ctypes.POINTER(I64)]
     L.tri_get_failed_units.argtypes = [P, P, P, I32, ctypes.POINTER(I32)]
     L.tri_decode_attention.argtypes = [P, ctypes.POINTER(tri_kv), P, P, P]
@@ -79,7 +80,8 @@ def _load():
     L.tri_status_str.argtypes = [ctypes.c_int]
     L.tri_status_str.restype = ctypes.c_char_p
     for fn in ("tri_create", "tri_destroy", "tri_calibrate_load", "tri_prune", "tri_prune_noalloc", "tri_score",
-               "tri_calibrate_estimate", "tri_append", "tri_get_error", "tri_set_tuning", "tri_set_offset_combine",
+               "tri_calibrate_estimate", "tri_append", "tri_append_advance", "tri_get_error", "tri_set_tuning",
+               "tri_set_offset_combine",
                "tri_get_failed_units", "tri_set_test_fault", "tri_decode_attention", "tri_set_score_engine",
                "tri_version"):
         getattr(L, fn).restype = ctypes.c_int
@@ -154,6 +156,10 @@ def tri_decode_attention(ctx, kv: tri_kv, q_ptr: int, out_ptr: int, stream: int)
 
 def tri_append(ctx, kv: tri_kv, k_new_ptr: int, v_new_ptr: int, pos_new_ptr: int, stream: int) -> int:
     return _lib.tri_append(ctx, ctypes.byref(kv), k_new_ptr, v_new_ptr, pos_new_ptr, stream)
+
+
+def tri_append_advance(ctx, kv: tri_kv, k_new_ptr: int, v_new_ptr: int, pos_ptr: int, stream: int) -> int:
+    return _lib.tri_append_advance(ctx, ctypes.byref(kv), k_new_ptr, v_new_ptr, pos_ptr, stream)
 
 
 def tri_get_error(ctx, stream: int):
@@ -326,9 +332,10 @@ class TriContext:
         return st
 
     def append(self, K, V, pos, lens, block_table, K_new, V_new, pos_new, lens_out="inplace", n_pages=None,
-               layer_begin=0, stream=None, check=True):
+               layer_begin=0, stream=None, check=True, advance=False):
         """Append one token per sequence to a paged cache (see make_kv for the layouts):
-        K_new, V_new bf16 [n_layers][batch][n_kv_heads][head_dim], pos_new int32 [batch]."""
+        K_new, V_new bf16 [n_layers][batch][n_kv_heads][head_dim], pos_new int32 [batch].
+        advance=True: tri_append_advance (pos_new then holds the next positions)."""
         if isinstance(lens_out, str):
             lens_out = lens
         kv = make_kv(K, V, pos, lens, lens_out, block_table, n_pages=n_pages, layer_begin=layer_begin)
@@ -336,10 +343,10 @@ class TriContext:
                             ("pos_new", pos_new, torch.int32)):
             if x.dtype != dt or not x.is_cuda or not x.is_contiguous():
                 raise ValueError(f"{name} must be a contiguous CUDA tensor of {dt}")
-        st = tri_append(self.handle, kv, K_new.data_ptr(), V_new.data_ptr(), pos_new.data_ptr(),
-                        _stream_handle(stream))
+        fn = tri_append_advance if advance else tri_append
+        st = fn(self.handle, kv, K_new.data_ptr(), V_new.data_ptr(), pos_new.data_ptr(), _stream_handle(stream))
         if check and st != TRI_OK:
-            raise TriError(st, "tri_append", tri_last_error(self.handle))
+            raise TriError(st, fn.__name__, tri_last_error(self.handle))
         return st
 
     def decode_attention(self, K, V, lens, q, out=None, block_table=None, n_pages=None, layer_begin=0,

@@ -57,6 +57,7 @@ def test_host_validation_without_device(lib):
     assert lib.tri_set_offset_combine(None, tri.TRI_OFFSETS_MAX) == tri.TRI_EINVAL
     assert tri.tri_calibrate_estimate(None, None, 1, 1, 1, 128, 0, None, None, None, None) == tri.TRI_EINVAL
     assert lib.tri_append(None, ctypes.byref(kv), None, None, None, None) == tri.TRI_EINVAL
+    assert lib.tri_append_advance(None, ctypes.byref(kv), None, None, None, None) == tri.TRI_EINVAL
     assert lib.tri_calibrate_load(None, 1, 1, 1, 64, ctypes.c_double(1e4), 0, None, None, None, None, 1) \
         == tri.TRI_EINVAL
     code = ctypes.c_int32(7)

@@ -202,6 +202,49 @@ def test_append_refuses_full_sequences():
     ctx.close()
 
 
+def test_append_advance_equals_append_then_position_update():
+    """tri_append_advance: the same rows as tri_append, and the positions advanced by one for the
+    sequences that accepted the token (a full sequence keeps its length and its position)."""
+    spec = ts.CacheSpec(name="adv", head_dim=128, group=2, n_kv_heads=2, n_layers=2, batch=3,
+                        rope_base=1e4, budget=16, offsets=(1, 2), positions="from_zero", lens=(1, 1, 1),
+                        page_size=16)
+    qm, qn, R, offsets = ts.make_stats(spec, 3)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(2, 2, 2, 128, 1e4, spec.layout, qm, qn, R, offsets)
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    steps = 5
+    new_k = torch.randn((steps, 2, 3, 2, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    new_v = torch.randn((steps, 2, 3, 2, 128), generator=gen, device="cuda").to(torch.bfloat16)
+    bt = torch.tensor([[0], [1], [2]], dtype=torch.int32, device="cuda")  # one page each: capacity 16
+
+    def fresh():
+        K = torch.zeros((2, 3, 2, 16, 128), dtype=torch.bfloat16, device="cuda")
+        # sequence 1 is two tokens from full, so it refuses the third step onwards
+        return K, K.clone(), torch.full((2, 3, 2, 16), -1, dtype=torch.int32, device="cuda"), \
+            torch.tensor([3, 14, 0], dtype=torch.int32, device="cuda"), \
+            torch.tensor([100, 200, 300], dtype=torch.int32, device="cuda")
+
+    K1, V1, P1, l1, t1 = fresh()
+    for i in range(steps):
+        before = l1.clone()
+        ctx.append(K1, V1, P1, l1, bt, new_k[i], new_v[i], t1, check=False)
+        t1.add_((l1 != before).to(torch.int32))  # the caller advances the accepted sequences
+    K2, V2, P2, l2, t2 = fresh()
+    for i in range(steps):
+        ctx.append(K2, V2, P2, l2, bt, new_k[i], new_v[i], t2, check=False, advance=True)
+    torch.cuda.synchronize()
+    assert l1.cpu().tolist() == l2.cpu().tolist() == [8, 16, 5]
+    assert t2.cpu().tolist() == [105, 202, 305]
+    assert torch.equal(t1, t2)
+    assert torch.equal(K1.view(torch.int16), K2.view(torch.int16))
+    assert torch.equal(V1.view(torch.int16), V2.view(torch.int16))
+    assert torch.equal(P1, P2)
+    assert int(P2[1, 1, 1, 15]) == 201 and int(P2[0, 2, 0, 4]) == 304
+    st, code, _ = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == 1  # TRI_DEV_LEN_GT_CAP (sequence 1)
+    ctx.close()
+
+
 def test_append_replays_from_a_cuda_graph():
     # the appends of a page span captured once and replayed give the same cache as the same
     # appends issued one by one
