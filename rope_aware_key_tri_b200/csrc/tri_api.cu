@@ -1058,13 +1058,27 @@ tri_status run_attend(tri_ctx *c, const tri_kv *kv, const void *q, float *out, v
     a.qscale = (float)(1.4426950408889634 / std::sqrt((double)c->D));
     a.status = c->d_status;
     a.wait_tries = c->wait_tries;
-    cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    fn<<<(unsigned)(n_units * cpu), tri::kAttThreads, tri::att_smem_bytes(c->D, c->G, nslot), cs>>>(a);
-    ce = cudaGetLastError();
+    // each launch a programmatic dependent of the one before on this stream (the validation, then
+    // the attention): its launch overlaps the previous grid's end; the kernels wait before they
+    // read what it wrote
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3((unsigned)(n_units * cpu));
+    cfg.blockDim = dim3((unsigned)tri::kAttThreads);
+    cfg.dynamicSmemBytes = tri::att_smem_bytes(c->D, c->G, nslot);
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
+    ce = cudaLaunchKernelEx(&cfg, fn, a);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(attend)");
     if (cpu > 1) {
-        comb<<<(unsigned)n_units, 256, 0, cs>>>(a);
-        ce = cudaGetLastError();
+        cfg.gridDim = dim3((unsigned)n_units);
+        cfg.blockDim = dim3(256u);
+        cfg.dynamicSmemBytes = 0;
+        ce = cudaLaunchKernelEx(&cfg, comb, a);
         if (ce != cudaSuccess) return cuda_fail(c, ce, "launch(attend combine)");
     }
     return TRI_OK;

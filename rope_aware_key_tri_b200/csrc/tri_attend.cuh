@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kAttThreads) tri_attend_kernel(const AttArgs a
     const int s = (unit / a.n_kv) % a.batch;
     const int lr = unit / (a.n_kv * a.batch);
     const int Hq = a.n_kv * G;
+    // a programmatic dependent of the validation kernel: its verdicts are read after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int N = __ldg(a.lens + s);
     if (__ldg(a.seq_bad + s) != 0 || N < 0 || N > a.cap_u) return;  // uniform: nothing is written
     const int per = ((N + a.cpu - 1) / a.cpu + kAttStageRows - 1) / kAttStageRows * kAttStageRows;
@@ -342,6 +344,8 @@ __global__ void __launch_bounds__(256) tri_attend_combine_kernel(const AttArgs a
     const int g = unit % a.n_kv;
     const int s = (unit / a.n_kv) % a.batch;
     const int lr = unit / (a.n_kv * a.batch);
+    // a programmatic dependent of the attention kernel: the partials are read after this
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int N = __ldg(a.lens + s);
     if (__ldg(a.seq_bad + s) != 0 || N < 0 || N > a.cap_u) return;
     const long long qrow = (((long long)lr * a.batch + s) * (a.n_kv * G) + (long long)g * G) * D;
