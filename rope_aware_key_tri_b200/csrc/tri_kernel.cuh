@@ -1289,6 +1289,22 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
             const unsigned buf_bytes = (unsigned)S2 * (4 * D + 4);
             const int wM = M / 32;
             const int q = count_ok ? gpre[wM] + __popc(gmask[wM] & ((1u << (M % 32)) - 1u)) : 0;
+            // Paged cache: the sequence's page ids in shared memory (the coefficient area, idle
+            // until the next unit), so that a moved row's address needs no global load. The
+            // block table row is read once; a table longer than the area keeps the global path.
+            const bool pt_smem = a.paged && a.page_shift >= 0 && a.max_pages <= G * D;  // uniform
+            const int *pt = reinterpret_cast<const int *>(coef_t);
+            if (pt_smem) {
+                for (int j = tid; j < a.max_pages; j += kThreads)
+                    reinterpret_cast<int *>(coef_t)[j] = __ldg(a.block_table + (long long)s * a.max_pages + j);
+                __syncthreads();
+            }
+            auto row_c = [&](int i) -> long long {
+                if (pt_smem)
+                    return (((long long)lr * a.n_pages + pt[i >> a.page_shift]) * a.n_kv + g) * (long long)a.page_size +
+                           (i & (a.page_size - 1));
+                return row_of(a, lr, s, g, i);
+            };
             // source slot of destination dst: the dst-th kept key
             auto source_of = [&](int dst) {
                 int lo = 0, hi = nwt;  // largest w with gpre[w] <= dst
@@ -1326,7 +1342,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                 for (int j = tid; j < nd; j += kThreads) sidx[j] = source_of(d0 + j);
                 __syncthreads();
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
-                    const long long srow = row_of(a, lr, s, g, sidx[rr]);
+                    const long long srow = row_c(sidx[rr]);
                     cp_async16(stK + (size_t)rr * D + qq * 8, a.K + srow * D + qq * 8);
                     cp_async16(stV + (size_t)rr * D + qq * 8, a.V + srow * D + qq * 8);
                     if (qq == 0) cp_async4(stP + rr, a.pos + srow);
@@ -1350,7 +1366,7 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                 const uint16_t *stV = stK + (size_t)S2 * D;
                 const int32_t *stP = reinterpret_cast<const int32_t *>(stV + (size_t)S2 * D);
                 for (int rr = warp * RPW + lane / LPR; rr < nd; rr += kWarps * RPW) {
-                    const long long drow = row_of(a, lr, s, g, d0 + rr);
+                    const long long drow = row_c(d0 + rr);
                     const uint4 xk = *reinterpret_cast<const uint4 *>(stK + (size_t)rr * D + qq * 8);
                     const uint4 xv = *reinterpret_cast<const uint4 *>(stV + (size_t)rr * D + qq * 8);
                     *reinterpret_cast<uint4 *>(a.K + drow * D + qq * 8) = xk;
