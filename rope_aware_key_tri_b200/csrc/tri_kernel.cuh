@@ -1299,7 +1299,9 @@ __global__ void __launch_bounds__(cta_threads(G, PRE), kMinBlocks) tri_fused_ker
                     reinterpret_cast<int *>(coef_t)[j] = __ldg(a.block_table + (long long)s * a.max_pages + j);
                 __syncthreads();
             }
+            // (the dense check first: the dense path keeps the one test it had)
             auto row_c = [&](int i) -> long long {
+                if (!a.paged) return (((long long)lr * a.batch + s) * a.n_kv + g) * (long long)a.cap_u + i;
                 if (pt_smem)
                     return (((long long)lr * a.n_pages + pt[i >> a.page_shift]) * a.n_kv + g) * (long long)a.page_size +
                            (i & (a.page_size - 1));
