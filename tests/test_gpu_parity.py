@@ -115,7 +115,7 @@ def test_cluster_sizes(cluster_size):
 
 
 @pytest.mark.parametrize("engine", ["cuda_cores", "tensor"])
-@pytest.mark.parametrize("page_size", [16, 64])
+@pytest.mark.parametrize("page_size", [16, 48, 64])  # 48: not a power of two (division path)
 def test_paged_permuted(page_size, engine):
     spec = _small("qwen3_32b_paged_ragged", n_layers=2, batch=3, lens=(700, 129, 513), page_size=page_size,
                   budget=128, cap=1024)
