@@ -140,7 +140,7 @@ def ncu_traffic(workload: str):
 
 def roofline_hbm(algorithmic_bytes: float, ms: float, traffic=None) -> dict:
     """HBM roofline block: achieved algorithmic GB/s against the measured copy peak (the
-    fraction the targets are judged on) and, for context, against the datasheet figure."""
+    fraction the bandwidth targets refer to) and, for context, against the datasheet figure."""
     peak, kind = measured_peak()
     achieved = algorithmic_bytes / (ms / 1e3) / 1e9
     return {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
