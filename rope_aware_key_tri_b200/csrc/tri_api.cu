@@ -1325,11 +1325,23 @@ tri_status append_impl(tri_ctx *c, const tri_kv *kv, const void *K_new, const vo
     a.pos_adv = advance ? const_cast<int32_t *>(pos_new) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
+    // a programmatic dependent of the launch before it on this stream (in a decode loop, the
+    // previous token's append): its launch overlaps that grid's end, and the kernel waits for
+    // it before its first memory access
+    cudaLaunchAttribute pdl[1];
+    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = dim3(blocks);
+    cfg.blockDim = dim3((unsigned)(tri::kAppendWarps * 32));
+    cfg.stream = st;
+    cfg.attrs = pdl;
+    cfg.numAttrs = 1;
     if (c->D == 128)
-        tri::tri_append_kernel<128><<<blocks, tri::kAppendWarps * 32, 0, st>>>(a);
+        ce = cudaLaunchKernelEx(&cfg, tri::tri_append_kernel<128>, a);
     else
-        tri::tri_append_kernel<64><<<blocks, tri::kAppendWarps * 32, 0, st>>>(a);
-    ce = cudaGetLastError();
+        ce = cudaLaunchKernelEx(&cfg, tri::tri_append_kernel<64>, a);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "append rows");
     return TRI_OK;
 }

@@ -8,7 +8,8 @@
 // generated tokens) every decode step appends the new token's key, value and position to each
 // (sequence, layer, KV head) unit of the paged cache, at slot lens[s]. One warp moves one unit's
 // K row and V row (16 bytes per lane) and its position; the last CTA to finish advances the
-// lengths of the sequences whose rows all went in (one launch per appended token).
+// lengths of the sequences whose rows all went in (one launch per appended token, each a
+// programmatic dependent of the launch before it).
 #pragma once
 
 #include <cuda_runtime.h>
@@ -41,6 +42,12 @@ __device__ __forceinline__ void append_record(unsigned long long *st, int code, 
 // One warp per unit (layer lr, sequence s, KV head g); the last CTA publishes the lengths.
 template <int D>
 __global__ void __launch_bounds__(kAppendWarps * 32) tri_append_kernel(const AppendArgs a) {
+    // launched as a programmatic dependent of the grid before it on the stream (usually the
+    // previous token's append, which writes the lengths, positions and counter read here):
+    // nothing is read before that grid has finished and its writes are visible; the next
+    // append may then be scheduled, so at most two appends are in flight
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    asm volatile("griddepcontrol.launch_dependents;");
     const int lane = threadIdx.x & 31;
     const long long unit = (long long)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
     const long long n_units = (long long)a.n_layers * a.batch * a.n_kv;
