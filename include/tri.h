@@ -191,10 +191,11 @@ TRI_API tri_status tri_calibrate_load(tri_ctx *ctx, int n_layers, int n_kv_heads
  * TRI_DEV_LEN_GT_CAP or TRI_DEV_BAD_PAGE): every unit of a sequence sees the same slot and
  * page, so a refused sequence receives no row. Needs the statistics loaded (for n_kv_heads
  * and head_dim).
- * One launch on `stream` (the last of its CTAs to finish writes lens_out), a programmatic
- * dependent of the work before it on the stream: its launch may overlap the end of the kernel
- * before it, but it reads and writes nothing until that kernel has finished, so stream order
- * holds as for a plain launch.
+ * One launch on `stream` (a cluster of CTAs per sequence, whose first CTA writes lens_out[s]
+ * after the cluster's barrier), a programmatic dependent of the work before it on the stream:
+ * its launch may overlap the end of the kernel before it, but it reads and writes nothing until
+ * that kernel has finished, so stream order holds as for a plain launch. tri_get_error reports
+ * a refused sequence s as unit s * n_kv_heads (its first layer and KV head).
  */
 TRI_API tri_status tri_append(tri_ctx *ctx, const tri_kv *kv, const void *K_new, const void *V_new,
                               const int32_t *pos_new, void *stream);

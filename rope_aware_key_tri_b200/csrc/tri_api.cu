@@ -59,12 +59,10 @@ struct tri_ctx {
     size_t att_part_bytes = 0;
     // device bookkeeping
     unsigned long long *d_status = nullptr;
-    // [0] CTAs of the fused kernel done, [1] its next free unit, [2] CTAs of tri_append done
+    // [0] CTAs of the fused kernel done, [1] its next free unit
     unsigned int *d_counter = nullptr;
     int32_t *d_seq_bad = nullptr;    // per-sequence verdict of the validation kernel
     int seq_bad_cap = 0;
-    int32_t *d_append_bad = nullptr; // per-sequence refusal flags of tri_append
-    int append_bad_cap = 0;
     unsigned *d_fail_count = nullptr;  // units left uncompacted by a unit-level failure ...
     int32_t *d_fail_units = nullptr;   // ... the first kFailCap of them
     // test hook (tri_set_test_fault): bounded waits' tries and the unit whose copy is withheld
@@ -1107,14 +1105,14 @@ tri_status tri_create(tri_ctx **out, int device) {
     c->sm_count = p.multiProcessorCount;
     c->max_smem_optin = (int)p.sharedMemPerBlockOptin;
     if (cudaMalloc(&c->d_status, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMalloc(&c->d_counter, 3 * sizeof(unsigned int)) != cudaSuccess ||
+        cudaMalloc(&c->d_counter, 2 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_count, sizeof(unsigned)) != cudaSuccess ||
         cudaMalloc(&c->d_fail_units, sizeof(int32_t) * kFailCap) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ENOMEM;
     }
     if (cudaMemset(c->d_status, 0, sizeof(unsigned long long)) != cudaSuccess ||
-        cudaMemset(c->d_counter, 0, 3 * sizeof(unsigned int)) != cudaSuccess ||
+        cudaMemset(c->d_counter, 0, 2 * sizeof(unsigned int)) != cudaSuccess ||
         cudaMemset(c->d_fail_count, 0, sizeof(unsigned)) != cudaSuccess) {
         tri_destroy(c);
         return TRI_ECUDA;
@@ -1130,7 +1128,6 @@ tri_status tri_destroy(tri_ctx *c) {
     cudaFree(c->d_status);
     cudaFree(c->d_counter);
     cudaFree(c->d_seq_bad);
-    cudaFree(c->d_append_bad);
     cudaFree(c->d_fail_count);
     cudaFree(c->d_fail_units);
     cudaFree(c->d_scratch);
@@ -1295,14 +1292,10 @@ tri_status append_impl(tri_ctx *c, const tri_kv *kv, const void *K_new, const vo
         !aligned(kv->pos, 4) || !aligned(kv->lens, 4) || !aligned(kv->lens_out, 4) || !aligned(pos_new, 4) ||
         !aligned(kv->block_table, 4))
         return TRI_EINVAL;
-    const long long n_units = (long long)kv->n_layers * kv->batch * c->Hkv;
-    if ((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps > 0x7fffffffLL) return TRI_EUNSUPPORTED;
+    const int cs = tri::append_cluster_size((long long)kv->n_layers * c->Hkv);
+    if ((long long)kv->batch * cs > 0x7fffffffLL) return TRI_EUNSUPPORTED;
     cudaError_t ce = cudaSetDevice(c->device);
     if (ce != cudaSuccess) return cuda_fail(c, ce, "cudaSetDevice");
-    {
-        const tri_status fs = ensure_flags(&c->d_append_bad, &c->append_bad_cap, kv->batch);
-        if (fs != TRI_OK) return fs;
-    }
     tri::AppendArgs a;
     a.K = static_cast<uint16_t *>(kv->K);
     a.V = static_cast<uint16_t *>(kv->V);
@@ -1319,25 +1312,26 @@ tri_status append_impl(tri_ctx *c, const tri_kv *kv, const void *K_new, const vo
     a.max_pages = kv->max_pages;
     a.n_pages = kv->n_pages;
     a.status = c->d_status;
-    a.seq_bad = c->d_append_bad;
     a.lens_out = kv->lens_out;
-    a.done = c->d_counter + 2;
     a.pos_adv = advance ? const_cast<int32_t *>(pos_new) : nullptr;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const unsigned blocks = (unsigned)((n_units + tri::kAppendWarps - 1) / tri::kAppendWarps);
-    // a programmatic dependent of the launch before it on this stream (in a decode loop, the
-    // previous token's append): its launch overlaps that grid's end, and the kernel waits for
-    // it before its first memory access
-    cudaLaunchAttribute pdl[1];
-    pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    pdl[0].val.programmaticStreamSerializationAllowed = 1;
+    // one cluster of cs CTAs per sequence; a programmatic dependent of the launch before it on
+    // this stream (in a decode loop, the previous token's append): its launch overlaps that
+    // grid's end, and the kernel waits for it before its first memory access
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg;
     std::memset(&cfg, 0, sizeof cfg);
-    cfg.gridDim = dim3(blocks);
+    cfg.gridDim = dim3((unsigned)(kv->batch * cs));
     cfg.blockDim = dim3((unsigned)(tri::kAppendWarps * 32));
     cfg.stream = st;
-    cfg.attrs = pdl;
-    cfg.numAttrs = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
     if (c->D == 128)
         ce = cudaLaunchKernelEx(&cfg, tri::tri_append_kernel<128>, a);
     else

@@ -6,18 +6,30 @@
 //
 // Between two prunes ([10100] §TriAttention方法 and [Summary] §方案设计 item 4: once every 128
 // generated tokens) every decode step appends the new token's key, value and position to each
-// (sequence, layer, KV head) unit of the paged cache, at slot lens[s]. One warp moves one unit's
-// K row and V row (16 bytes per lane) and its position; the last CTA to finish advances the
-// lengths of the sequences whose rows all went in (one launch per appended token, each a
-// programmatic dependent of the launch before it).
+// (sequence, layer, KV head) unit of the paged cache, at slot lens[s]. One cluster of CTAs per
+// sequence: every unit of a sequence sees the same slot and the same page, so one thread per CTA
+// looks them up, the warps move the units' K and V rows (16 bytes per lane) and positions, and
+// after a cluster barrier the cluster's first CTA publishes the new length (one launch per
+// appended token, each a programmatic dependent of the launch before it).
 #pragma once
 
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 namespace tri {
 
-constexpr int kAppendWarps = 8;  // units per CTA
+namespace cg = cooperative_groups;
+
+constexpr int kAppendWarps = 16;      // warps per CTA (512 threads)
+constexpr int kAppendMaxCluster = 8;  // CTAs per sequence, at most (the portable cluster size)
+constexpr int kAppendBatch = 4;       // units per warp whose rows are loaded before any is stored
+
+// CTAs per sequence for n_units_per_seq = n_layers * n_kv units: one unit per warp where possible.
+inline int append_cluster_size(long long n_units_per_seq) {
+    const long long need = (n_units_per_seq + kAppendWarps - 1) / kAppendWarps;
+    return (int)(need < 1 ? 1 : need > kAppendMaxCluster ? kAppendMaxCluster : need);
+}
 
 struct AppendArgs {
     uint16_t *K, *V;              // paged pools [n_layers][n_pages][n_kv][page_size][D]
@@ -29,8 +41,6 @@ struct AppendArgs {
     const int32_t *block_table;   // [batch][max_pages]
     int batch, n_kv, n_layers, page_size, max_pages, n_pages;
     unsigned long long *status;   // first device-detected problem
-    int32_t *seq_bad;             // [batch] refused sequences
-    unsigned *done;               // completed-CTA counter (zero between launches)
     int32_t *pos_adv;             // pos_new itself, advanced by one for the accepted sequences (or null)
 };
 
@@ -39,71 +49,91 @@ __device__ __forceinline__ void append_record(unsigned long long *st, int code, 
     atomicCAS(st, 0ull, v);
 }
 
-// One warp per unit (layer lr, sequence s, KV head g); the last CTA publishes the lengths.
+// Grid: batch clusters of cs CTAs (launched with that cluster size); cluster c appends to
+// sequence c. Unit u = lr * n_kv + g of the sequence goes to warp u mod (cs * kAppendWarps) of
+// the cluster, in batches of kAppendBatch units per warp.
 template <int D>
 __global__ void __launch_bounds__(kAppendWarps * 32) tri_append_kernel(const AppendArgs a) {
     // launched as a programmatic dependent of the grid before it on the stream (usually the
-    // previous token's append, which writes the lengths, positions and counter read here):
-    // nothing is read before that grid has finished and its writes are visible; the next
-    // append may then be scheduled, so at most two appends are in flight
+    // previous token's append, which writes the lengths and positions read here): nothing is
+    // read before that grid has finished and its writes are visible; the next append may then
+    // be scheduled, so at most two appends are in flight
     asm volatile("griddepcontrol.wait;" ::: "memory");
     asm volatile("griddepcontrol.launch_dependents;");
-    const int lane = threadIdx.x & 31;
-    const long long unit = (long long)blockIdx.x * kAppendWarps + (threadIdx.x >> 5);
-    const long long n_units = (long long)a.n_layers * a.batch * a.n_kv;
-    if (unit < n_units) {
-        const int g = (int)(unit % a.n_kv);
-        const int s = (int)((unit / a.n_kv) % a.batch);
-        const int lr = (int)(unit / ((long long)a.n_kv * a.batch));
-        const int n = a.lens[s];  // plain load: lens_out may be lens, written at the end of this launch
+    cg::cluster_group cluster = cg::this_cluster();
+    const int cs = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    const int s = (int)(blockIdx.x / cs);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int per_seq = a.n_layers * a.n_kv;
+    const int stride = cs * kAppendWarps;
+    constexpr int PIECES = D / 8;  // 16-byte pieces per row; lane p < 2 PIECES moves piece p of K then V
+    const bool mover = lane < 2 * PIECES;
+    const bool isv = lane >= PIECES;
+    const int q = isv ? lane - PIECES : lane;
+
+    uint4 x[kAppendBatch];
+    auto load = [&](int u0) {
+#pragma unroll
+        for (int k = 0; k < kAppendBatch; ++k) {
+            const int u = u0 + k * stride;
+            if (mover && u < per_seq) {
+                const long long src = ((long long)(u / a.n_kv) * a.batch + s) * a.n_kv + u % a.n_kv;
+                x[k] = __ldg(reinterpret_cast<const uint4 *>((isv ? a.V_new : a.K_new) + src * D) + q);
+            }
+        }
+    };
+    int u0 = rank * kAppendWarps + warp;
+    load(u0);  // the source rows do not depend on the slot: in flight during the lookup
+
+    __shared__ int n_s, page_s, bad_s, p_s;
+    if (threadIdx.x == 0) {
+        const int n = a.lens[s];  // plain loads: lens_out may be lens, pos_adv is pos_new
         const long long cap = (long long)a.page_size * a.max_pages;
-        int page = -1;
-        int bad = 0;
+        int page = -1, bad = 0;
         if (n < 0 || n >= cap) {
             bad = 1;  // TRI_DEV_LEN_GT_CAP: no slot left for the new token
         } else {
             page = __ldg(a.block_table + (long long)s * a.max_pages + n / a.page_size);
             if (page < 0 || page >= a.n_pages) bad = 2;  // TRI_DEV_BAD_PAGE: the page is not allocated
         }
+        n_s = n;
+        page_s = page;
+        bad_s = bad;
+        p_s = a.pos_new[s];
+    }
+    __syncthreads();
+    const int n = n_s, bad = bad_s;
+    if (!bad) {
+        const long long page_row = (long long)page_s * a.n_kv;
+        const int slot = n % a.page_size;
+        for (;;) {
+#pragma unroll
+            for (int k = 0; k < kAppendBatch; ++k) {
+                const int u = u0 + k * stride;
+                if (u < per_seq) {
+                    const long long row =
+                        (((long long)(u / a.n_kv) * a.n_pages * a.n_kv + page_row) + u % a.n_kv) * a.page_size + slot;
+                    if (mover) reinterpret_cast<uint4 *>((isv ? a.V : a.K) + row * D)[q] = x[k];
+                    if (lane == 0) a.pos[row] = p_s;
+                }
+            }
+            u0 += kAppendBatch * stride;
+            if (u0 >= per_seq) break;
+            load(u0);
+        }
+    }
+    // every CTA of the cluster has read lens[s] and pos_new[s]: the length (and, when asked, the
+    // next position) can be published; a refused sequence keeps both
+    cluster.sync();
+    if (rank == 0 && threadIdx.x == 0) {
         if (bad) {
-            if (lane == 0) {
-                append_record(a.status, bad, unit);
-                atomicExch(a.seq_bad + s, 1);
-            }
+            append_record(a.status, bad, (long long)s * a.n_kv);  // unit (layer 0, s, head 0)
+            a.lens_out[s] = n;
         } else {
-            const long long row =
-                (((long long)lr * a.n_pages + page) * a.n_kv + g) * a.page_size + n % a.page_size;
-            const long long src = ((long long)lr * a.batch + s) * a.n_kv + g;
-            constexpr int PIECES = D / 8;  // 16-byte pieces per row
-            for (int p = lane; p < 2 * PIECES; p += 32) {
-                const bool isv = p >= PIECES;
-                const int q = isv ? p - PIECES : p;
-                const uint4 x = __ldg(reinterpret_cast<const uint4 *>((isv ? a.V_new : a.K_new) + src * D) + q);
-                reinterpret_cast<uint4 *>((isv ? a.V : a.K) + row * D)[q] = x;
-            }
-            if (lane == 0) a.pos[row] = __ldg(a.pos_new + s);
+            a.lens_out[s] = n + 1;
+            if (a.pos_adv) a.pos_adv[s] = p_s + 1;  // the next token's position
         }
-    }
-    // lens_out[s] = lens[s] + 1 for every sequence whose rows all went in (and, when asked, its
-    // next position pos_new[s] + 1); refused sequences keep both and their flag is cleared for
-    // the next call. Done by the last CTA to finish, after every CTA has read the lengths and
-    // positions and raised its flags.
-    __shared__ int last_s;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        last_s = atomicAdd(a.done, 1u) == gridDim.x - 1;
-    }
-    __syncthreads();
-    if (last_s) {
-        __threadfence();
-        for (int s = threadIdx.x; s < a.batch; s += blockDim.x) {
-            const int n = a.lens[s];
-            const int refused = atomicExch(a.seq_bad + s, 0);
-            a.lens_out[s] = refused ? n : n + 1;
-            if (a.pos_adv && !refused) a.pos_adv[s] += 1;  // the next token's position
-        }
-        if (threadIdx.x == 0) atomicExch(a.done, 0u);
     }
 }
 }  // namespace tri
