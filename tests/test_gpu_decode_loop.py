@@ -289,3 +289,51 @@ def test_append_replays_from_a_cuda_graph():
     assert torch.equal(P1, P2) and torch.equal(t1, t2)
     assert int(P1[0, 1, 0, 0]) == 40 and int(P1[1, 5, 1, 15]) == 75
     ctx.close()
+
+
+@pytest.mark.parametrize("n_layers,n_kv,d", [(72, 8, 128), (5, 8, 64)])
+def test_append_many_units_per_sequence(n_layers, n_kv, d):
+    """Sequences with many (layer, KV head) units: 576 units per sequence take clusters of 8
+    CTAs and two batches of loads per warp, 40 units take clusters of 3. Every unit of an
+    accepted sequence receives its rows and position at slot lens[s] and nothing else changes;
+    a sequence whose slot lands in an unallocated page is refused whole; lens (also lens_out)
+    and the positions advance for the accepted ones only."""
+    PS_, batch = 16, 4
+    spec = ts.CacheSpec(name="wide", head_dim=d, group=2, n_kv_heads=n_kv, n_layers=n_layers, batch=batch,
+                        rope_base=1e4, budget=16, offsets=(1, 2), positions="from_zero",
+                        lens=(1,) * batch, page_size=PS_)
+    qm, qn, R, offsets = ts.make_stats(spec, 4)
+    ctx = tri.TriContext(0)
+    ctx.calibrate_load(n_layers, n_kv, 2, d, 1e4, spec.layout, qm, qn, R, offsets)
+    gen = torch.Generator(device="cuda").manual_seed(9)
+    n_pages = 7
+    K = torch.randn((n_layers, n_pages, n_kv, PS_, d), generator=gen, device="cuda").to(torch.bfloat16)
+    V = torch.randn((n_layers, n_pages, n_kv, PS_, d), generator=gen, device="cuda").to(torch.bfloat16)
+    P = torch.randint(0, 1000, (n_layers, n_pages, n_kv, PS_), generator=gen, device="cuda", dtype=torch.int32)
+    new_k = torch.randn((n_layers, batch, n_kv, d), generator=gen, device="cuda").to(torch.bfloat16)
+    new_v = torch.randn((n_layers, batch, n_kv, d), generator=gen, device="cuda").to(torch.bfloat16)
+    # sequence 1's slot 16 is in its second page, which is not allocated: refused
+    bt_h = [[0, 1], [2, -1], [3, 4], [5, 6]]
+    lens_h = [5, 16, 31, 0]
+    pos_h = [100, 200, 300, 400]
+    bt = torch.tensor(bt_h, dtype=torch.int32, device="cuda")
+    lens = torch.tensor(lens_h, dtype=torch.int32, device="cuda")
+    pos = torch.tensor(pos_h, dtype=torch.int32, device="cuda")
+    K_exp, V_exp, P_exp = K.clone(), V.clone(), P.clone()
+    for s in (0, 2, 3):
+        n = lens_h[s]
+        page = bt_h[s][n // PS_]
+        K_exp[:, page, :, n % PS_] = new_k[:, s]
+        V_exp[:, page, :, n % PS_] = new_v[:, s]
+        P_exp[:, page, :, n % PS_] = pos_h[s]
+    ctx.append(K, V, P, lens, bt, new_k, new_v, pos, check=False, advance=True)
+    torch.cuda.synchronize()
+    st, code, unit = ctx.get_error()
+    assert st == tri.TRI_EDEVICE and code == 2  # TRI_DEV_BAD_PAGE (sequence 1)
+    assert unit == 1 * n_kv                       # reported as (layer 0, sequence 1, head 0)
+    assert lens.cpu().tolist() == [6, 16, 32, 1]
+    assert pos.cpu().tolist() == [101, 200, 301, 401]
+    assert torch.equal(K.view(torch.int16), K_exp.view(torch.int16))
+    assert torch.equal(V.view(torch.int16), V_exp.view(torch.int16))
+    assert torch.equal(P, P_exp)
+    ctx.close()
